@@ -1,0 +1,386 @@
+"""Benchmark of the fused attention forward (libattn) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of the workload
+(for the FP8 workload: Hadamard rotation + quantisation of Q, K, V and the
+FP8 attention).  The default workload is the GPT-2-shaped case
+(B=8, H=12, N=1024, d=64, causal, bf16).  Rank 0 prints one JSON line.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronisation; each step's kernels are timed with CUDA events on the
+launching stream, and the L2 cache (126 MB) is flushed by writing a 256 MB
+buffer between steps, outside the timed events.  Multi-GPU runs are weak
+scaling: every rank runs its own copy of the workload (independent batches,
+no data-path collective) and the job time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on this machine's host cores on a
+bounded sample of the same workload (the reference arm; there is no other
+implementation of these pages to run).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import attn_inputs as gen  # noqa: E402
+
+METRIC = "attn fwd TFLOP/s (4·B·H·N²·d, causal/2) and % of B200 dense BF16 peak"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def workloads():
+    w = {
+        "tiny": dict(B=1, Hq=1, Hkv=1, N=128, d=64, causal=False, dtype="bf16"),
+        "gpt2": dict(B=8, Hq=12, Hkv=12, N=1024, d=64, causal=True, dtype="bf16"),
+        "gqa": dict(B=4, Hq=32, Hkv=8, N=4096, d=128, causal=True, dtype="bf16"),
+        "mqa": dict(B=4, Hq=32, Hkv=1, N=4096, d=128, causal=True, dtype="bf16"),
+        "d256": dict(B=2, Hq=8, Hkv=8, N=4096, d=256, causal=False, dtype="bf16"),
+        "fp8": dict(B=4, Hq=16, Hkv=16, N=8192, d=128, causal=False, dtype="fp8"),
+    }
+    for n in (512, 1024, 2048, 4096, 8192, 16384):
+        for c in (False, True):
+            w[f"sweep{n}{'c' if c else ''}"] = dict(B=16384 // n, Hq=16, Hkv=16, N=n, d=128, causal=c, dtype="bf16")
+    return w
+
+
+def flops(cfg) -> float:
+    f = 4.0 * cfg["B"] * cfg["Hq"] * cfg["N"] * cfg["N"] * cfg["d"]
+    return f / 2 if cfg["causal"] else f
+
+
+def describe(name, cfg):
+    return (f"{name}: B={cfg['B']} Hq={cfg['Hq']} Hkv={cfg['Hkv']} N={cfg['N']} d={cfg['d']} "
+            f"{'causal' if cfg['causal'] else 'non-causal'} {cfg['dtype']}")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(bf16=j["bf16_tflops"], hbm=j["hbm_gbs"], src="measured")
+    return dict(bf16=1590.0, hbm=6650.0, src="fallback")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, dev_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self.stop_ev, self.thread = period_s, threading.Event(), None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(dev_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self.nv = None
+
+    def _run(self):
+        while not self.stop_ev.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:  # noqa: BLE001
+            pass
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.thread is not None:
+            self.stop_ev.set()
+            self.thread.join()
+            self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def make_inputs(cfg, seed=gen.BASE_SEED):
+    outl = cfg["dtype"] == "fp8"
+    return gen.qkv_bf16(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["N"], cfg["N"], cfg["d"], seed=seed, outliers=outl)
+
+
+def _row_flops(cfg, rows):
+    i = rows % cfg["N"]
+    keys = np.minimum(cfg["N"], i + 1) if cfg["causal"] else np.full(rows.shape, cfg["N"])
+    return float(np.sum(4.0 * cfg["d"] * keys))
+
+
+def oracle_sample(cfg, qb, kb, vb, target_s: float, n_rows: int | None = None, seed: int = 0):
+    """Times the fp64 oracle on a bounded uniform sample of query rows (all their
+    keys).  With n_rows None the sample is grown until one run takes about
+    target_s.  Returns (TFLOP/s, description, seconds, n_rows)."""
+    import oracle
+    B, Hq, N, d = cfg["B"], cfg["Hq"], cfg["N"], cfg["d"]
+    total_rows = B * Hq * N
+    q, k, v = gen.bf16_bits_to_f64(qb), gen.bf16_bits_to_f64(kb), gen.bf16_bits_to_f64(vb)
+    rng = np.random.default_rng(seed)
+    n = min(total_rows, n_rows or 256)
+    while True:
+        rows = np.sort(rng.choice(total_rows, size=n, replace=False))
+        t0 = time.perf_counter()
+        oracle.attn_fwd_rows(q, k, v, cfg["causal"], 1.0 / math.sqrt(d), rows)
+        dt = time.perf_counter() - t0
+        if n_rows is not None or dt >= 0.8 * target_s or n == total_rows:
+            break
+        n = min(total_rows, max(n * 2, int(n * target_s / max(dt, 1e-3))))
+    tf = _row_flops(cfg, rows) / dt / 1e12
+    desc = f"{n} of {total_rows} query rows (uniform sample), all their keys, fp64"
+    return tf, desc, dt, n
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, cfg, name):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    qb, kb, vb = make_inputs(cfg)
+    per_step = max(0.5, min(10.0, 60.0 / max(1, args.steps + args.warmup)))
+    _, _, _, n_rows = oracle_sample(cfg, qb, kb, vb, per_step)  # size the per-step sample
+    vals = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        tf, desc, dt, _ = oracle_sample(cfg, qb, kb, vb, per_step, n_rows=n_rows, seed=i)
+        if i >= args.warmup:
+            vals.append(tf)
+    v = float(statistics.median(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": flops(cfg) / (v * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(name, cfg), "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, cfg, name):
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_140_b200 as ea
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    B, Hq, Hkv, N, d, causal = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["N"], cfg["d"], cfg["causal"]
+    scale = 1.0 / math.sqrt(d)
+    fp8 = cfg["dtype"] == "fp8"
+
+    qb, kb, vb = make_inputs(cfg, seed=gen.BASE_SEED + 1000 * rank)
+    host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (qb, kb, vb)]
+    q, k, v = (h.to(dev) for h in host)
+    o = torch.empty((B, N, Hq, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    o_host = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+    lse_host = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    if fp8:
+        signs = torch.from_numpy(gen.hadamard_signs(gen.BASE_SEED + 3, d)).to(dev)
+        q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+        k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
+        v8 = torch.empty(v.shape, dtype=torch.uint8, device=dev)
+        desc = torch.empty(3, dtype=torch.float32, device=dev)
+        ws = torch.empty(3 * ea.attn_hadamard_quant_fp8_workspace_bytes(), dtype=torch.uint8, device=dev)
+        wsb = ea.attn_hadamard_quant_fp8_workspace_bytes()
+
+        def step(qq, kk, vv):
+            ea.attn_hadamard_quant_fp8(qq, q8, desc.data_ptr(), ws.data_ptr(), B * N * Hq, d, signs, stream)
+            ea.attn_hadamard_quant_fp8(kk, k8, desc.data_ptr() + 4, ws.data_ptr() + wsb, B * N * Hkv, d, signs,
+                                       stream)
+            ea.attn_hadamard_quant_fp8(vv, v8, desc.data_ptr() + 8, ws.data_ptr() + 2 * wsb, B * N * Hkv, d, None,
+                                       stream)
+            ea.attn_fwd_fp8(q8, k8, v8, o, lse, B, Hq, Hkv, N, N, d, causal, scale, desc.data_ptr(),
+                            desc.data_ptr() + 4, desc.data_ptr() + 8, stream)
+        launches_per_step = 7  # 3 x (amax + quantise) + attention
+    else:
+        def step(qq, kk, vv):
+            ea.attn_fwd(qq, kk, vv, o, lse, B, Hq, Hkv, N, N, d, causal, scale, ea.ATTN_BF16, stream)
+        launches_per_step = 1
+
+    for _ in range(max(3, args.warmup)):
+        step(q, k, v)
+    torch.cuda.synchronize()
+    if args.steps <= 0:  # size the timed region to about 1.5 s (L2 flush included)
+        w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0.record(stream)
+        for i in range(5):
+            flush.fill_(float(i))
+            step(q, k, v)
+        w1.record(stream)
+        torch.cuda.synchronize()
+        per = w0.elapsed_time(w1) / 5 * 1e-3
+        t = torch.tensor([int(min(20000, max(20, 1.5 / per)))], device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        args.steps = int(t.item())
+    rc, word = ea.attn_get_last_device_error(stream)
+    if rc != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    kstarts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] if fp8 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            starts[i].record(stream)
+            if fp8:
+                ea.attn_hadamard_quant_fp8(q, q8, desc.data_ptr(), ws.data_ptr(), B * N * Hq, d, signs, stream)
+                ea.attn_hadamard_quant_fp8(k, k8, desc.data_ptr() + 4, ws.data_ptr() + wsb, B * N * Hkv, d, signs,
+                                           stream)
+                ea.attn_hadamard_quant_fp8(v, v8, desc.data_ptr() + 8, ws.data_ptr() + 2 * wsb, B * N * Hkv, d,
+                                           None, stream)
+                kstarts[i].record(stream)
+                ea.attn_fwd_fp8(q8, k8, v8, o, lse, B, Hq, Hkv, N, N, d, causal, scale, desc.data_ptr(),
+                                desc.data_ptr() + 4, desc.data_ptr() + 8, stream)
+            else:
+                step(q, k, v)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kern_ms = [s.elapsed_time(e) for s, e in zip(kstarts, ends)] if fp8 else step_ms
+    total_ms = float(sum(step_ms))
+    rc, word = ea.attn_get_last_device_error(stream)
+    if rc != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+
+    # end to end through the C ABI with host buffers: H2D inputs, kernel(s), D2H outputs
+    e2e_steps = max(3, min(args.steps, 50))
+    e_st = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e_en = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    dq, dk, dv = (torch.empty_like(x) for x in (q, k, v))
+    for i in range(e2e_steps):
+        e_st[i].record(stream)
+        dq.copy_(host[0], non_blocking=True)
+        dk.copy_(host[1], non_blocking=True)
+        dv.copy_(host[2], non_blocking=True)
+        step(dq, dk, dv)
+        o_host.copy_(o, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+        e_en[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_st, e_en)))
+
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.destroy_process_group()
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+    if rank != 0:
+        return 0
+
+    peaks = load_peaks()
+    f = flops(cfg)
+    value = f * args.steps * world / (total_ms * 1e-3) / 1e12
+    e2e_value = f * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    kern_avg_s = float(np.mean(kern_ms)) * 1e-3
+    achieved = f / kern_avg_s / 1e12
+    peak = peaks["bf16"] * (2.0 if fp8 else 1.0)
+    traffic = TRAFFIC.get(name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3" if fp8 else "bf16", "data": "synthetic",
+        "config": {"workload": describe(name, cfg), "global_batch": cfg["B"] * world, "seq_len": N,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed between steps (256 MB write)",
+                   "pct_of_peak": round(100.0 * value / world / peak, 2)},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peaks['src']} {'bf16 x2 (fp8 nominal ratio)' if fp8 else 'bf16'}",
+                     "kernel": "attn_fwd_kernel"},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in host)),
+                "d2h_bytes_per_step": int(o.numel() * o.element_size() + lse.numel() * lse.element_size())},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        tf, desc, dt, _ = oracle_sample(cfg, qb, kb, vb, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                                "sample": desc + f"; {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# dram bytes (read + write) per launch of the attention kernel from an ncu capture of
+# the same kernel; null until taken for the current kernel
+TRAFFIC: dict = {}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=0, help="timed steps (0 = enough for about 1.5 s)")
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gpt2", choices=sorted(workloads()))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = workloads()[args.workload]
+    if args.impl == "reference":
+        if args.steps <= 0:
+            args.steps = 3
+        return run_reference(args, cfg, args.workload)
+    return run_ours(args, cfg, args.workload)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,157 @@
+"""Python binding of libattn, the sm_100a fused exact-attention forward.
+
+Each function here has the name of a C entry point in ``include/attn.h`` and
+only marshals arguments (tensor -> device pointer, stream -> handle) before
+calling into ``libattn.so``; every step of the computation runs in the CUDA
+kernels.  There is no fallback: if the shared library is missing or cannot be
+loaded, importing this package raises.
+
+``attention()`` is a convenience wrapper that allocates the outputs with
+PyTorch and calls ``attn_fwd``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = [
+    "ATTN_BF16", "ATTN_FP8_E4M3", "AttnError", "attn_fwd", "attn_fwd_fp8", "attn_hadamard_quant_fp8",
+    "attn_hadamard_quant_fp8_workspace_bytes", "attn_get_last_device_error", "attn_status_string",
+    "attn_kv_tile_count", "attn_tile_kind", "attn_debug_unsatisfied_wait", "attention", "lib_path", "EXPORTS",
+]
+
+ATTN_BF16 = 0
+ATTN_FP8_E4M3 = 1
+STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_MISALIGNED",
+          4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_DEVICE_TIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libattn.so")
+
+# every symbol include/attn.h declares
+EXPORTS = (
+    "attn_fwd", "attn_fwd_fp8", "attn_hadamard_quant_fp8", "attn_hadamard_quant_fp8_workspace_bytes",
+    "attn_get_last_device_error", "attn_status_string", "attn_kv_tile_count", "attn_tile_kind",
+    "attn_debug_unsatisfied_wait",
+)
+
+if not os.path.exists(lib_path):
+    raise ImportError(f"libattn.so is not built ({lib_path}); run `python exact_attention_140_b200/build.py` "
+                      "or __graft_entry__.build()")
+_lib = ctypes.CDLL(lib_path)
+
+_vp, _I, _LL, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
+_lib.attn_fwd.argtypes = [_vp] * 5 + [_I] * 7 + [_F, _I, _vp]
+_lib.attn_fwd.restype = _I
+_lib.attn_fwd_fp8.argtypes = [_vp] * 5 + [_I] * 7 + [_F, _vp, _vp, _vp, _vp]
+_lib.attn_fwd_fp8.restype = _I
+_lib.attn_hadamard_quant_fp8.argtypes = [_vp, _vp, _vp, _vp, _LL, _I, _vp, _vp]
+_lib.attn_hadamard_quant_fp8.restype = _I
+_lib.attn_hadamard_quant_fp8_workspace_bytes.argtypes = []
+_lib.attn_hadamard_quant_fp8_workspace_bytes.restype = _LL
+_lib.attn_get_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint)]
+_lib.attn_get_last_device_error.restype = _I
+_lib.attn_status_string.argtypes = [_I]
+_lib.attn_status_string.restype = ctypes.c_char_p
+_lib.attn_kv_tile_count.argtypes = [_I] * 6
+_lib.attn_kv_tile_count.restype = _I
+_lib.attn_tile_kind.argtypes = [_I] * 7
+_lib.attn_tile_kind.restype = _I
+_lib.attn_debug_unsatisfied_wait.argtypes = [_LL, _vp]
+_lib.attn_debug_unsatisfied_wait.restype = _I
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({attn_status_string(status)})")
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(rc: int, where: str, raise_on_error: bool):
+    if rc != 0 and raise_on_error:
+        raise AttnError(rc, where)
+    return rc
+
+
+def attn_status_string(status: int) -> str:
+    return _lib.attn_status_string(int(status)).decode()
+
+
+def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype=ATTN_BF16, stream=None,
+             raise_on_error=True):
+    rc = _lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, int(causal),
+                       float(scale), int(dtype), _stream(stream))
+    return _check(rc, "attn_fwd", raise_on_error)
+
+
+def attn_fwd_fp8(q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, descale_q, descale_k, descale_v,
+                 stream=None, raise_on_error=True):
+    rc = _lib.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, int(causal),
+                           float(scale), _ptr(descale_q), _ptr(descale_k), _ptr(descale_v), _stream(stream))
+    return _check(rc, "attn_fwd_fp8", raise_on_error)
+
+
+def attn_hadamard_quant_fp8_workspace_bytes() -> int:
+    return int(_lib.attn_hadamard_quant_fp8_workspace_bytes())
+
+
+def attn_hadamard_quant_fp8(x, x8, descale, workspace, rows, d, signs=None, stream=None, raise_on_error=True):
+    rc = _lib.attn_hadamard_quant_fp8(_ptr(x), _ptr(x8), _ptr(descale), _ptr(workspace), int(rows), int(d),
+                                      _ptr(signs), _stream(stream))
+    return _check(rc, "attn_hadamard_quant_fp8", raise_on_error)
+
+
+def attn_get_last_device_error(stream=None):
+    """Returns (status, raw error word); synchronises the stream."""
+    w = ctypes.c_uint(0)
+    rc = _lib.attn_get_last_device_error(_stream(stream), ctypes.byref(w))
+    return rc, w.value
+
+
+def attn_kv_tile_count(row0, row1, Nq, Nk, bn, causal) -> int:
+    return int(_lib.attn_kv_tile_count(row0, row1, Nq, Nk, bn, int(causal)))
+
+
+def attn_tile_kind(row0, row1, kt, Nq, Nk, bn, causal) -> int:
+    return int(_lib.attn_tile_kind(row0, row1, kt, Nq, Nk, bn, int(causal)))
+
+
+def attn_debug_unsatisfied_wait(limit_ns: int, stream=None, raise_on_error=True):
+    rc = _lib.attn_debug_unsatisfied_wait(int(limit_ns), _stream(stream))
+    return _check(rc, "attn_debug_unsatisfied_wait", raise_on_error)
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None, return_lse: bool = True, stream=None):
+    """O, LSE for torch tensors q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d] (bf16, CUDA, contiguous)."""
+    import torch
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("attention() takes bf16 tensors; use attn_fwd_fp8 for e4m3")
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if return_lse else None
+    attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, ATTN_BF16, stream)
+    return (o, lse) if return_lse else o

@@ -1,0 +1,327 @@
+// attn_api.cu -- the C ABI of libattn (declared in include/attn.h): argument
+// checks, TMA descriptor encoding, choice of kernel instantiation, launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "attn.h"
+#include "attn_fwd_kernel.cuh"
+#include "fp8_prep.cuh"
+#include "tiles.h"
+
+namespace attn {
+namespace {
+
+__device__ unsigned int g_err_word;     // device error word (bounded waits that ran out)
+__device__ float g_unit_descale = 1.0f;  // descale used when attn_fwd is given e4m3 inputs
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+
+struct DeviceState {
+  bool init = false;
+  int status = ATTN_OK;
+  unsigned int* err = nullptr;
+  int num_sms = 0;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+unsigned long long timeout_ns() {
+  static unsigned long long v = [] {
+    const char* e = std::getenv("ATTN_WAIT_TIMEOUT_NS");
+    if (e == nullptr) return kDefaultTimeoutNs;
+    const unsigned long long x = std::strtoull(e, nullptr, 10);
+    return x > 0 ? x : kDefaultTimeoutNs;
+  }();
+  return v;
+}
+
+// Per-device setup: checks for an sm_100 device and finds the error word.
+int device_state(int* dev_out, DeviceState** st_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.init) {
+    st.init = true;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      st.status = ATTN_ERR_CUDA;
+    } else if (major != 10 || minor != 0) {
+      st.status = ATTN_ERR_UNSUPPORTED;  // built for sm_100a only
+    } else if (cudaGetSymbolAddress(reinterpret_cast<void**>(&st.err), g_err_word) != cudaSuccess) {
+      st.status = ATTN_ERR_CUDA;
+    }
+    if (st.status == ATTN_OK && g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        st.status = ATTN_ERR_CUDA;
+      else
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+  }
+  *dev_out = dev;
+  *st_out = &st;
+  return st.status;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 4-D tiled map over a [B, N, H, d] tensor: dims (d, H, N, B), box
+// (128 bytes of d, 1 head, rows, 1), 128-byte swizzle, zero fill out of range.
+int encode_bnhd(CUtensorMap* m, const void* ptr, bool fp8, int B, int N, int H, int d, int rows) {
+  const cuuint64_t es = fp8 ? 1 : 2;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)H * d * es, (cuuint64_t)N * H * d * es};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / es), 1u, (cuuint32_t)rows, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  const CUresult r = g_encode(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                              const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+__global__ void empty_rows_kernel(__nv_bfloat16* o, float* lse, long long n_o, long long n_lse) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_o; i += (long long)gridDim.x * blockDim.x)
+    o[i] = __float2bfloat16(0.f);
+  if (lse != nullptr)
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_lse;
+         i += (long long)gridDim.x * blockDim.x)
+      lse[i] = -INFINITY;
+}
+
+__global__ void unsatisfied_wait_kernel(unsigned int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t mbar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(ptx::smem_u32(&mbar), 1);  // one arrival expected; none ever comes
+    abort_flag = 0u;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtx wc{&abort_flag, err, limit_ns};
+    wait_bar(ptx::smem_u32(&mbar), 0u, wc, kSiteProbe);
+  }
+  __syncthreads();
+}
+
+template <class Cfg>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+               int Nk, float scale, const float* dq, const float* dk, const float* dv, DeviceState* st,
+               cudaStream_t stream) {
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Cfg::SMEM_BYTES) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tq, tk, tv;
+  if (encode_bnhd(&tq, q, Cfg::FP8, B, Nq, Hq, Cfg::D, Cfg::BM) != ATTN_OK ||
+      encode_bnhd(&tk, k, Cfg::FP8, B, Nk, Hkv, Cfg::D, Cfg::BN) != ATTN_OK ||
+      encode_bnhd(&tv, v, Cfg::FP8, B, Nk, Hkv, Cfg::D, Cfg::BN) != ATTN_OK)
+    return ATTN_ERR_CUDA;
+  FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.group = Hq / Hkv;
+  p.n_qblocks = (Nq + Cfg::BM * Cfg::NQT - 1) / (Cfg::BM * Cfg::NQT);
+  p.sl2 = scale * 1.4426950408889634f;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.err = st->err;
+  p.timeout_ns = timeout_ns();
+  const dim3 grid((unsigned)p.n_qblocks, (unsigned)Hq, (unsigned)B);
+  attn_fwd_kernel<Cfg><<<grid, Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, int BN, int NQT, int KST, int VST, bool FP8>
+int launch_causal(bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                  int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
+                  DeviceState* st, cudaStream_t s) {
+  if (causal)
+    return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, true, FP8>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk,
+                                                                dv, st, s);
+  return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, false, FP8>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk,
+                                                               dv, st, s);
+}
+
+int check_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                 int Nk, int causal, float scale) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || Hq == 0 || Nq == 0) return -1;  // nothing to compute
+  if (Hkv == 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (o == nullptr || (Nk > 0 && (q == nullptr || k == nullptr || v == nullptr))) return ATTN_ERR_INVALID_ARG;
+  if (B > 65535 || Hq > 65535) return ATTN_ERR_UNSUPPORTED;  // grid y / z limits
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+  return ATTN_OK;
+}
+
+int fill_empty(void* o, float* lse, int B, int Hq, int Nq, int d, cudaStream_t s) {
+  const long long n_o = (long long)B * Nq * Hq * d, n_lse = (long long)B * Hq * Nq;
+  empty_rows_kernel<<<256, 256, 0, s>>>(reinterpret_cast<__nv_bfloat16*>(o), lse, n_o, n_lse);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case ATTN_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int attn_kv_tile_count(int row0, int row1, int Nq, int Nk, int bn, int causal) {
+  if (row0 < 0 || row1 < row0 || Nq < 0 || Nk < 0 || bn <= 0 || (causal != 0 && causal != 1)) return -1;
+  return kv_tile_count(row0, row1, Nq, Nk, bn, causal != 0);
+}
+
+int attn_tile_kind(int row0, int row1, int kt, int Nq, int Nk, int bn, int causal) {
+  if (row0 < 0 || row1 < row0 || kt < 0 || Nq < 0 || Nk < 0 || bn <= 0 || (causal != 0 && causal != 1)) return -1;
+  return tile_kind(row0, row1, kt, Nq, Nk, bn, causal != 0);
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk,
+             int d, int causal, float scale, int dtype, void* stream) {
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if (dtype == ATTN_FP8_E4M3) {
+    // e4m3 inputs with unit scales: attn_fwd_fp8 with descales read from a
+    // device constant 1.0 (argument checks come before any CUDA call)
+    int rc = check_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, scale);
+    if (rc == -1) return ATTN_OK;
+    if (rc != ATTN_OK) return rc;
+    if (d != 128) return ATTN_ERR_UNSUPPORTED;
+    int dev = 0;
+    DeviceState* st = nullptr;
+    if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
+    void* one = nullptr;
+    if (cudaGetSymbolAddress(&one, g_unit_descale) != cudaSuccess) return ATTN_ERR_CUDA;
+    const float* u = static_cast<const float*>(one);
+    return attn_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, u, u, u, stream);
+  }
+  int rc = check_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, scale);
+  if (rc == -1) return ATTN_OK;
+  if (rc != ATTN_OK) return rc;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  int dev = 0;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
+  const bool c = causal != 0;
+  switch (d) {
+    case 64: return launch_causal<64, 128, 2, 3, 3, false>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
+                                                          nullptr, nullptr, st, s);
+    case 128: return launch_causal<128, 128, 2, 2, 2, false>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
+                                                            nullptr, nullptr, st, s);
+    default: return launch_causal<256, 64, 1, 2, 2, false>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
+                                                          nullptr, nullptr, st, s);
+  }
+}
+
+int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                 int Nk, int d, int causal, float scale, const float* descale_q, const float* descale_k,
+                 const float* descale_v, void* stream) {
+  int rc = check_common(q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, causal, scale);
+  if (rc == -1) return ATTN_OK;
+  if (rc != ATTN_OK) return rc;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Nk > 0 && (descale_q == nullptr || descale_k == nullptr || descale_v == nullptr)) return ATTN_ERR_INVALID_ARG;
+  int dev = 0;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
+  return launch_causal<128, 128, 2, 3, 3, true>(causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, scale, descale_q,
+                                                descale_k, descale_v, st, s);
+}
+
+long long attn_hadamard_quant_fp8_workspace_bytes(void) { return 256; }
+
+int attn_hadamard_quant_fp8(const void* x, void* x8, float* descale, void* workspace, long long rows, int d,
+                            const float* signs, void* stream) {
+  if (rows < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != kPrepD) return ATTN_ERR_UNSUPPORTED;
+  if (x == nullptr || x8 == nullptr || descale == nullptr || workspace == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x8) || !aligned16(workspace) || !aligned16(signs) ||
+      (reinterpret_cast<uintptr_t>(descale) & 3u) != 0)
+    return ATTN_ERR_MISALIGNED;
+  int dev = 0, rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int* amax = static_cast<unsigned int*>(workspace);
+  if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), s) != cudaSuccess) return ATTN_ERR_CUDA;
+  const long long blocks_needed = (rows + kPrepWarps - 1) / kPrepWarps;
+  const long long cap = (long long)st->num_sms * 16;
+  const unsigned grid = (unsigned)(blocks_needed < 1 ? 1 : (blocks_needed < cap ? blocks_needed : cap));
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  fp8_amax_kernel<<<grid, 32 * kPrepWarps, 0, s>>>(xb, rows, signs, amax);
+  fp8_quant_kernel<<<grid, 32 * kPrepWarps, 0, s>>>(xb, rows, signs, amax, static_cast<uint8_t*>(x8), descale);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_get_last_device_error(void* stream, unsigned int* detail) {
+  int dev = 0, rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpy(&word, st->err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (word != 0 && cudaMemcpy(st->err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (detail != nullptr) *detail = word;
+  return word != 0 ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
+}
+
+int attn_debug_unsatisfied_wait(long long limit_ns, void* stream) {
+  if (limit_ns <= 0 || limit_ns > 10000000000ll) return ATTN_ERR_INVALID_ARG;
+  int dev = 0, rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
+  unsatisfied_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(st->err, (unsigned long long)limit_ns);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,506 @@
+// attn_fwd_kernel.cuh -- fused exact-attention forward for sm_100a.
+//
+// One CTA computes NQT query tiles of 128 rows for one (batch, query head).
+// It walks the key/value tiles of that head once, keeping the output
+// accumulator on chip, so neither the score matrix nor partial outputs ever
+// reach HBM (page "FlashAttention (SV)": tiling, online softmax and operator
+// fusion; the query-tile-outer loop order is the one page "FlashAttention-4
+// 震撼发布" credits to FlashAttention-2's re-partitioned work).
+//
+// Warp roles (warp specialisation, page "FlashAttention-3 — 闪电注意力-3",
+// section 1, recast for tcgen05):
+//   warps 0 .. 4*NQT-1  softmax: warp w serves query tile w/4 and TMEM lanes
+//                       32*(w%4) .. +31, so thread = one query row;
+//   warp 4*NQT          TMA producer: Q tiles once, then K_j and V_j through
+//                       KST / VST-stage shared-memory rings (section 2: the
+//                       next block is fetched while the current one computes);
+//   warp 4*NQT+1        MMA issuer: one thread issues every tcgen05.mma;
+//                       also allocates and frees tensor memory.
+//
+// Tensor memory (128 lanes x 512 fp32 columns): per query tile t, SB score
+// buffers S of BN columns (P overwrites S in place: BN/2 columns of packed
+// bf16, or BN/4 of e4m3) and the output accumulator O of D columns.  With two
+// query tiles (NQT = 2) the tensor core alternates between them, so one
+// tile's softmax runs under the other's matrix products (the ping-pong idea
+// of section 1); with one tile the score buffer is doubled instead (SB = 2)
+// so S_{j+1} = Q K_{j+1}^T runs under the softmax of S_j.
+//
+// Per key tile j and query tile t:
+//   S   = Q_t K_j^T                          (tcgen05, SS operands, fp32 in TMEM)
+//   m_b = rowmax(scale*log2e * S)            (masked on partial tiles)
+//   if m_b > m_ref + TAU: rescale O_t and l by 2^(m_ref - m_b), m_ref = m_b
+//   P   = 2^(scale*log2e * S - m_ref);  l += rowsum(P)
+//   O_t += P V_j                             (tcgen05, A = P from TMEM)
+// The reference max only moves when the block max exceeds it by more than
+// TAU (lazy rescaling; page "FlashAttention-4震撼发布", the new online
+// softmax that skips most output rescalings).  The result is the same for any
+// TAU because the reference cancels in O = acc / l; TAU = 8 bounds P by 2^8.
+// Epilogue: O = O_t / l (bf16), LSE = ln2 * (m_ref + log2 l).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "tiles.h"
+
+namespace attn {
+
+struct FwdParams {
+  void* o;          // [B, Nq, Hq, D] bf16
+  float* lse;       // [B, Hq, Nq] fp32 or nullptr
+  int B, Hq, Hkv, Nq, Nk;
+  int group;        // Hq / Hkv
+  int n_qblocks;    // ceil(Nq / (128 * NQT))
+  float sl2;        // scale * log2(e)
+  const float* dq;  // FP8 descales (device scalars), nullptr for bf16
+  const float* dk;
+  const float* dv;
+  unsigned int* err;            // device error word
+  unsigned long long timeout_ns;
+};
+
+constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
+
+template <int D_, int BN_, int NQT_, int KST_, int VST_, bool CAUSAL_, bool FP8_>
+struct FwdCfg {
+  static constexpr int D = D_, BN = BN_, NQT = NQT_, KST = KST_, VST = VST_;
+  static constexpr bool CAUSAL = CAUSAL_, FP8 = FP8_;
+  static constexpr int BM = 128;
+  static constexpr int SB = NQT == 1 ? 2 : 1;
+  static constexpr int ELEM = FP8 ? 1 : 2;
+  static constexpr int NCH = D * ELEM / 128;  // 128-byte column chunks per row
+  static constexpr int BOXE = 128 / ELEM;     // elements per chunk row
+  static constexpr uint32_t CH_Q = BM * 128;  // bytes of one chunk of a Q tile
+  static constexpr uint32_t CH_KV = BN * 128;
+  static constexpr uint32_t QT_BYTES = CH_Q * NCH;
+  static constexpr uint32_t KV_BYTES = CH_KV * NCH;
+  static constexpr int KSTEP = FP8 ? 32 : 16;  // reduction depth of one MMA
+  static constexpr int QK_STEPS = D / KSTEP;
+  static constexpr int PV_STEPS = BN / KSTEP;
+  static constexpr int P_COLS = BN * ELEM / 4;
+  static constexpr int O_COL0 = NQT * SB * BN;
+  static constexpr int TMEM_USED = O_COL0 + NQT * D;
+  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
+  static_assert(TMEM_USED <= 512, "tensor memory has 512 columns");
+  static_assert(D % 64 == 0 && NCH >= 1, "head size");
+  static_assert(BN % 32 == 0 && BN <= 256, "key tile");
+  // barriers
+  static constexpr int B_QFULL = 0;
+  static constexpr int B_KFULL = B_QFULL + NQT;
+  static constexpr int B_KEMPTY = B_KFULL + KST;
+  static constexpr int B_VFULL = B_KEMPTY + KST;
+  static constexpr int B_VEMPTY = B_VFULL + VST;
+  static constexpr int B_SFULL = B_VEMPTY + VST;
+  static constexpr int B_PFULL = B_SFULL + NQT * SB;
+  static constexpr int B_ODONE = B_PFULL + NQT * SB;
+  static constexpr int B_DRAIN = B_ODONE + NQT;
+  static constexpr int NBAR = B_DRAIN + 1;
+  // shared memory (offsets from a 1024-byte aligned base)
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = OFF_Q + NQT * QT_BYTES;
+  static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_V + VST * KV_BYTES;
+  static constexpr uint32_t OFF_SLOT = OFF_BAR + NBAR * 8;
+  static constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
+  static constexpr uint32_t SMEM_BYTES = OFF_ABORT + 4 + 1024;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per block");
+  // warps
+  static constexpr int SM_WARPS = 4 * NQT;
+  static constexpr int TMA_WARP = SM_WARPS;
+  static constexpr int MMA_WARP = SM_WARPS + 1;
+  static constexpr int NTHREADS = 32 * (SM_WARPS + 2);
+  static constexpr uint32_t IDESC_QK = ptx::idesc<FP8>(128, BN, false);
+  static constexpr uint32_t IDESC_PV = ptx::idesc<FP8>(128, D, true);
+};
+
+// Wait sites recorded in the device error word.
+enum : uint32_t {
+  kSiteQ = 1, kSiteKFull, kSiteVFull, kSiteKEmpty, kSiteVEmpty, kSiteSFull, kSitePFull,
+  kSiteODone, kSiteDrain, kSiteProbe
+};
+
+struct WaitCtx {
+  volatile uint32_t* abort;
+  unsigned int* err;
+  unsigned long long timeout_ns;
+};
+
+// Bounded mbarrier wait: true when the phase with `parity` has completed;
+// false after the time limit (recording the site in the error word and
+// raising the block's abort flag) or when another role already aborted.
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, const WaitCtx& c, uint32_t site) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*c.abort) return false;
+    if (ptx::globaltimer() - t0 > c.timeout_ns) {
+      *c.abort = 1u;
+      const uint32_t blk = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+      atomicOr(c.err, 1u | (site << 8) | ((blk & 0xFFFFu) << 16));
+      return false;
+    }
+  }
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::NTHREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  constexpr int BM = Cfg::BM, BN = Cfg::BN, D = Cfg::D, NQT = Cfg::NQT, SB = Cfg::SB;
+  constexpr int KST = Cfg::KST, VST = Cfg::VST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
+  const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw_u32);
+  auto bar = [&](int i) -> uint32_t { return sbase + Cfg::OFF_BAR + 8u * (uint32_t)i; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sgen + Cfg::OFF_ABORT);
+  const WaitCtx wc{abort_flag, p.err, p.timeout_ns};
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = p.n_qblocks - 1 - (int)blockIdx.x;  // longest causal blocks first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kh = h / p.group;
+  const int q0 = qb * BM * NQT;
+  int n_kv[NQT];
+  int nmax = 0;
+#pragma unroll
+  for (int t = 0; t < NQT; ++t) {
+    n_kv[t] = kv_tile_count(q0 + t * BM, q0 + (t + 1) * BM, p.Nq, p.Nk, BN, Cfg::CAUSAL);
+    nmax = n_kv[t] > nmax ? n_kv[t] : nmax;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < NQT; ++t) ptx::mbar_init(bar(Cfg::B_QFULL + t), 1);
+    for (int s = 0; s < KST; ++s) {
+      ptx::mbar_init(bar(Cfg::B_KFULL + s), 1);
+      ptx::mbar_init(bar(Cfg::B_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < VST; ++s) {
+      ptx::mbar_init(bar(Cfg::B_VFULL + s), 1);
+      ptx::mbar_init(bar(Cfg::B_VEMPTY + s), 1);
+    }
+    for (int i = 0; i < NQT * SB; ++i) {
+      ptx::mbar_init(bar(Cfg::B_SFULL + i), 1);
+      ptx::mbar_init(bar(Cfg::B_PFULL + i), 128);
+    }
+    for (int t = 0; t < NQT; ++t) ptx::mbar_init(bar(Cfg::B_ODONE + t), 1);
+    ptx::mbar_init(bar(Cfg::B_DRAIN), 1);
+    *abort_flag = 0u;
+    ptx::fence_mbar_init();
+  }
+  if (warp == Cfg::TMA_WARP && lane == 0) {
+    ptx::prefetch_tmap(&tmQ);
+    ptx::prefetch_tmap(&tmK);
+    ptx::prefetch_tmap(&tmV);
+  }
+  if (warp == Cfg::MMA_WARP) {
+    ptx::tmem_alloc(sbase + Cfg::OFF_SLOT, Cfg::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sgen + Cfg::OFF_SLOT);
+
+  if (warp < Cfg::SM_WARPS) {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2, wq = warp & 3;
+    const int row0 = q0 + t * BM;
+    const int row = row0 + wq * 32 + lane;
+    const int nt = n_kv[t];
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t o_taddr = tmem + lane_off + (uint32_t)(Cfg::O_COL0 + t * D);
+    float sl2 = p.sl2;
+    if constexpr (Cfg::FP8) sl2 *= __ldg(p.dq) * __ldg(p.dk);
+    const long long vend = vis_end(row, p.Nq, p.Nk, Cfg::CAUSAL);
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int si = t * SB + (j % SB);
+      ok = wait_bar(bar(Cfg::B_SFULL + si), (uint32_t)((j / SB) & 1), wc, kSiteSFull);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const uint32_t s_taddr = tmem + lane_off + (uint32_t)(si * BN);
+      uint32_t sr[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c)
+        ptx::tmem_ld32(s_taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+      ptx::tmem_wait_ld();
+      float s[BN];
+#pragma unroll
+      for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(sr[c]);
+      const bool partial = tile_kind(row0, row0 + BM, j, p.Nq, p.Nk, BN, Cfg::CAUSAL) == kTilePartial;
+      float m_blk;
+      if (partial) {
+        const long long k0 = (long long)j * BN;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const float x = (k0 + c < vend) ? s[c] * sl2 : -INFINITY;
+          s[c] = x;
+          mx = fmaxf(mx, x);
+        }
+        m_blk = mx;
+      } else {
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < BN; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        if (sl2 < 0.f) {  // a negative scale turns the row max into the row min
+          mx = s[0];
+#pragma unroll
+          for (int c = 1; c < BN; ++c) mx = fminf(mx, s[c]);
+        }
+        m_blk = mx * sl2;
+      }
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_blk > m_ref + kTau) {
+        alpha = ptx::ex2(m_ref - m_blk);  // 0 when m_ref = -inf
+        resc = (m_ref != -INFINITY);
+        m_ref = m_blk;
+        l *= alpha;
+      }
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // exponentiate, accumulate the row sum and pack P in one pass, so each
+      // score register dies as soon as its packed weight exists
+      float l0 = 0.f, l1 = 0.f;
+      uint32_t pk[Cfg::P_COLS];
+      constexpr int PER = Cfg::FP8 ? 4 : 2;  // weights per 32-bit TMEM column
+#pragma unroll
+      for (int c = 0; c < Cfg::P_COLS; ++c) {
+        float e[PER];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+          const float x = s[PER * c + u];
+          e[u] = ptx::ex2(partial ? (x - m_use) : fmaf(x, sl2, -m_use));
+        }
+        if constexpr (Cfg::FP8) {
+          l0 += e[0] + e[1];
+          l1 += e[2] + e[3];
+          pk[c] = ptx::pack_e4m3x4(e[0], e[1], e[2], e[3]);
+        } else {
+          l0 += e[0];
+          l1 += e[1];
+          pk[c] = ptx::pack_bf16x2(e[0], e[1]);
+        }
+      }
+      l += l0 + l1;
+#pragma unroll
+      for (int c = 0; c < Cfg::P_COLS / 32; ++c)
+        ptx::tmem_st32(s_taddr + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * c]));
+      if constexpr (Cfg::P_COLS % 32 == 16) ptx::tmem_st16(s_taddr + (Cfg::P_COLS / 32) * 32, &pk[Cfg::P_COLS - 16]);
+      ptx::tmem_wait_st();
+      if (j > 0) {
+        // PV(t, j-1) must be complete before P(t, j) is released (and before
+        // O_t is rescaled).  Observing every o_done phase in order keeps the
+        // barrier within one phase of this thread's view, so parity waits are
+        // unambiguous.
+        ok = wait_bar(bar(Cfg::B_ODONE + t), (uint32_t)((j - 1) & 1), wc, kSiteODone);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+        ptx::tc_fence_after();
+        const float a = resc ? alpha : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(o_taddr + 32 * c, r);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * a);
+          ptx::tmem_st32(o_taddr + 32 * c, r);
+        }
+        ptx::tmem_wait_st();
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(Cfg::B_PFULL + si));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && nt > 0) {
+      ok = wait_bar(bar(Cfg::B_ODONE + t), (uint32_t)((nt - 1) & 1), wc, kSiteODone);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      ptx::tc_fence_after();
+      const bool store = row < p.Nq;
+      float inv = l > 0.f ? 1.f / l : 0.f;
+      if constexpr (Cfg::FP8) inv *= __ldg(p.dv);
+      __nv_bfloat16* orow =
+          reinterpret_cast<__nv_bfloat16*>(p.o) + (((long long)b * p.Nq + row) * p.Hq + h) * (long long)D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        if (nt > 0) {
+          ptx::tmem_ld32(o_taddr + 32 * c, r);
+          ptx::tmem_wait_ld();
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = nt > 0 ? ptx::pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv)
+                        : 0u;
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+      if (store && p.lse != nullptr) {
+        const float lse = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        p.lse[((long long)b * p.Hq + h) * p.Nq + row] = lse;
+      }
+    }
+  } else if (warp == Cfg::TMA_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int k_issued[KST], v_issued[VST];
+#pragma unroll
+      for (int s = 0; s < KST; ++s) k_issued[s] = 0;
+#pragma unroll
+      for (int s = 0; s < VST; ++s) v_issued[s] = 0;
+      bool q_issued[NQT];
+#pragma unroll
+      for (int t = 0; t < NQT; ++t) {
+        q_issued[t] = n_kv[t] > 0;
+        if (!q_issued[t]) continue;
+        const uint32_t fb = bar(Cfg::B_QFULL + t);
+        ptx::mbar_arrive_expect_tx(fb, Cfg::QT_BYTES);
+#pragma unroll
+        for (int c = 0; c < Cfg::NCH; ++c)
+          ptx::tma_load_4d(sbase + Cfg::OFF_Q + t * Cfg::QT_BYTES + c * Cfg::CH_Q, &tmQ, fb, c * Cfg::BOXE, h,
+                           q0 + t * BM, b);
+      }
+      for (int j = 0; j < nmax; ++j) {
+        const int ks = j % KST;
+        if (j >= KST && !wait_bar(bar(Cfg::B_KEMPTY + ks), (uint32_t)(((j / KST) - 1) & 1), wc, kSiteKEmpty))
+          break;
+        {
+          const uint32_t fb = bar(Cfg::B_KFULL + ks);
+          ptx::mbar_arrive_expect_tx(fb, Cfg::KV_BYTES);
+#pragma unroll
+          for (int c = 0; c < Cfg::NCH; ++c)
+            ptx::tma_load_4d(sbase + Cfg::OFF_K + ks * Cfg::KV_BYTES + c * Cfg::CH_KV, &tmK, fb, c * Cfg::BOXE,
+                             kh, j * BN, b);
+          ++k_issued[ks];
+        }
+        const int vs = j % VST;
+        if (j >= VST && !wait_bar(bar(Cfg::B_VEMPTY + vs), (uint32_t)(((j / VST) - 1) & 1), wc, kSiteVEmpty))
+          break;
+        {
+          const uint32_t fb = bar(Cfg::B_VFULL + vs);
+          ptx::mbar_arrive_expect_tx(fb, Cfg::KV_BYTES);
+#pragma unroll
+          for (int c = 0; c < Cfg::NCH; ++c)
+            ptx::tma_load_4d(sbase + Cfg::OFF_V + vs * Cfg::KV_BYTES + c * Cfg::CH_KV, &tmV, fb, c * Cfg::BOXE,
+                             kh, j * BN, b);
+          ++v_issued[vs];
+        }
+      }
+      // Every issued copy must land before the block may exit (no-op in the
+      // normal path, where the consumers have already seen them all).
+#pragma unroll
+      for (int t = 0; t < NQT; ++t)
+        if (q_issued[t]) wait_bar(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
+#pragma unroll
+      for (int s = 0; s < KST; ++s)
+        if (k_issued[s] > 0) wait_bar(bar(Cfg::B_KFULL + s), (uint32_t)((k_issued[s] - 1) & 1), wc, kSiteKFull);
+#pragma unroll
+      for (int s = 0; s < VST; ++s)
+        if (v_issued[s] > 0) wait_bar(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
+    }
+  } else {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+#pragma unroll
+      for (int t = 0; t < NQT && ok; ++t)
+        if (n_kv[t] > 0) ok = wait_bar(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
+      ptx::tc_fence_after();
+      const uint32_t q_s = sbase + Cfg::OFF_Q, k_s = sbase + Cfg::OFF_K, v_s = sbase + Cfg::OFF_V;
+      for (int j = 0; ok && j <= nmax; ++j) {
+        const bool has_k = j < nmax, has_v = j >= 1;
+        if (has_k) {
+          ok = wait_bar(bar(Cfg::B_KFULL + j % KST), (uint32_t)((j / KST) & 1), wc, kSiteKFull);
+          if (!ok) break;
+        }
+        if (has_v) {
+          ok = wait_bar(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc, kSiteVFull);
+          if (!ok) break;
+        }
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int t = 0; t < NQT; ++t) {
+          auto issue_qk = [&]() {
+            if (!(has_k && j < n_kv[t])) return;
+            const uint32_t d_t = tmem + (uint32_t)((t * SB + j % SB) * BN);
+            const uint32_t qa = q_s + t * Cfg::QT_BYTES;
+            const uint32_t kb = k_s + (j % KST) * Cfg::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < Cfg::QK_STEPS; ++kk) {
+              const uint32_t off = (uint32_t)kk * 32u;  // bytes along the reduction dim
+              const uint32_t ch = off / 128u, in = off % 128u;
+              const uint64_t ad = ptx::sdesc_sw128(qa + ch * Cfg::CH_Q + in, 16u, 1024u);
+              const uint64_t bd = ptx::sdesc_sw128(kb + ch * Cfg::CH_KV + in, 16u, 1024u);
+              ptx::mma_ss<Cfg::FP8>(d_t, ad, bd, Cfg::IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+            ptx::tc_commit(bar(Cfg::B_SFULL + t * SB + j % SB));
+          };
+          auto issue_pv = [&]() -> bool {
+            const int jj = j - 1;
+            if (!(has_v && jj < n_kv[t])) return true;
+            const int si = t * SB + jj % SB;
+            if (!wait_bar(bar(Cfg::B_PFULL + si), (uint32_t)((jj / SB) & 1), wc, kSitePFull)) return false;
+            ptx::tc_fence_after();
+            const uint32_t d_t = tmem + (uint32_t)(Cfg::O_COL0 + t * D);
+            const uint32_t a_t = tmem + (uint32_t)(si * BN);
+            const uint32_t vb = v_s + (jj % VST) * Cfg::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < Cfg::PV_STEPS; ++kk) {
+              const uint64_t bd = ptx::sdesc_sw128(vb + (uint32_t)kk * Cfg::KSTEP * 128u, Cfg::CH_KV, 1024u);
+              ptx::mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV,
+                                    (jj > 0 || kk > 0) ? 1u : 0u);
+            }
+            ptx::tc_commit(bar(Cfg::B_ODONE + t));
+            return true;
+          };
+          if (SB == 2) {
+            issue_qk();
+            ok = issue_pv();
+          } else {
+            ok = issue_pv();
+            if (ok) issue_qk();
+          }
+          if (!ok) break;
+        }
+        if (!ok) break;
+        if (has_k) ptx::tc_commit(bar(Cfg::B_KEMPTY + j % KST));
+        if (has_v) ptx::tc_commit(bar(Cfg::B_VEMPTY + (j - 1) % VST));
+      }
+      // All issued MMAs must finish before tensor memory is freed.
+      ptx::tc_commit(bar(Cfg::B_DRAIN));
+      wait_bar(bar(Cfg::B_DRAIN), 0u, wc, kSiteDrain);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == Cfg::MMA_WARP) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

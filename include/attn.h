@@ -1,0 +1,165 @@
+/*
+ * attn.h -- C ABI of libattn, the B200 (sm_100a) fused exact-attention forward.
+ *
+ * The operation (page "FlashAttention (SV)", section "Problematik med
+ * standard-attention", the attention formula; tiled with the online softmax
+ * of section "Online-beräkning av Softmax" and fused into one kernel as in
+ * section "Sammanslagning av operationer till en enda CUDA-kärna"):
+ *
+ *   S = scale * Q K^T  (+ causal mask),   O = softmax(S) V,
+ *   LSE[i] = ln sum_j exp(S[i, j])        (natural log of the scaled scores)
+ *
+ * Head sizes 64, 128 and 256 and grouped/multi-query heads follow page
+ * "FlashAttention-4震撼发布：性能再攀新高" (the FlashAttention-2 list: head
+ * size up to 256, MQA and GQA).  The FP8 entry points follow page
+ * "FlashAttention-3 — 闪电注意力-3", section 3 (FP8 with incoherent
+ * processing: rotate Q and K by a random orthogonal Hadamard matrix, then
+ * quantise).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers:  every tensor pointer is a DEVICE pointer owned by the caller
+ *            (for example torch.empty(...).data_ptr()).  The library keeps no
+ *            reference after the call returns and allocates no device memory
+ *            for the caller's data.  Tensor pointers must be 16-byte aligned
+ *            (the tiles are moved by the Tensor Memory Accelerator).
+ * Layout:    Q and O are [B, Nq, Hq, d]; K and V are [B, Nk, Hkv, d]; all
+ *            contiguous row-major with d innermost.  LSE is [B, Hq, Nq] fp32.
+ * Heads:     query head h reads key/value head h / (Hq / Hkv); Hq % Hkv == 0
+ *            (Hkv == Hq is multi-head, Hkv == 1 multi-query).
+ * Causal:    bottom-right aligned.  Query row i sees key j iff
+ *            j <= i + (Nk - Nq).  With Nq == Nk this is j <= i.  A row that
+ *            sees no key (only when Nq > Nk) gets O = 0 and LSE = -inf.
+ * Stream:    `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *            stream).  Every call is asynchronous on that stream and returns
+ *            after the launch; device results are ready when the stream is.
+ * Errors:    argument errors are returned synchronously as attn_status_t and
+ *            nothing is launched.  A launch failure returns ATTN_ERR_CUDA.
+ *            Every device-side wait is bounded: a wait that runs out records
+ *            an error word on the device instead of hanging; read it with
+ *            attn_get_last_device_error().
+ * Threads:   all entry points are thread-safe.
+ * Empty:     B == 0, Hq == 0 or Nq == 0 is a no-op returning ATTN_OK.  Nk == 0
+ *            gives O = 0 and LSE = -inf for every row.
+ */
+#ifndef LIBATTN_ATTN_H_
+#define LIBATTN_ATTN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,    /* null pointer, negative size, Hq % Hkv != 0, non-finite scale */
+    ATTN_ERR_UNSUPPORTED = 2,    /* head size or dtype not built, or not an sm_100 device */
+    ATTN_ERR_MISALIGNED = 3,     /* a tensor pointer is not 16-byte aligned */
+    ATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
+    ATTN_ERR_DEVICE_TIMEOUT = 5  /* a device-side wait ran out (see attn_get_last_device_error) */
+} attn_status_t;
+
+typedef enum {
+    ATTN_BF16 = 0,     /* Q, K, V in bfloat16 */
+    ATTN_FP8_E4M3 = 1  /* Q, K, V in OCP FP8 E4M3 with unit scales */
+} attn_dtype_t;
+
+/*
+ * attn_fwd -- fused attention forward.
+ *   q      [B, Nq, Hq, d]  bf16 (or e4m3 bytes when dtype == ATTN_FP8_E4M3)
+ *   k, v   [B, Nk, Hkv, d] same dtype as q
+ *   o      [B, Nq, Hq, d]  bf16 output (always bf16)
+ *   lse    [B, Hq, Nq]     fp32 output, natural log; may be NULL to skip it
+ *   d      64, 128 or 256 for bf16; 128 for FP8
+ *   causal 0 or 1
+ *   scale  finite multiplier of Q K^T (1/sqrt(d) for the usual attention)
+ *   dtype  attn_dtype_t
+ * Returns ATTN_OK or an error code; see the conventions above.
+ */
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+             int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+             int dtype, void *stream);
+
+/*
+ * attn_fwd_fp8 -- FP8 E4M3 attention forward with per-tensor scales.
+ * Page "FlashAttention-3 — 闪电注意力-3", section 3: the inputs are quantised
+ * (Q and K after the Hadamard rotation, see attn_hadamard_quant_fp8) and the
+ * products run on FP8 tensor cores.  The real inputs are q8*dq, k8*dk, v8*dv:
+ *   S = scale * dq * dk * (q8 k8^T);  P = softmax weights rounded to E4M3;
+ *   O = dv * (P v8) / rowsum,  bf16.
+ *   q8, k8, v8   e4m3 bytes, layouts as attn_fwd; d must be 128
+ *   descale_q/k/v  DEVICE pointers to one fp32 each (dq, dk, dv), as written
+ *                  by attn_hadamard_quant_fp8, so no host synchronisation is
+ *                  needed between quantisation and attention
+ * Returns ATTN_OK or an error code.
+ */
+int attn_fwd_fp8(const void *q8, const void *k8, const void *v8, void *o, float *lse,
+                 int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                 const float *descale_q, const float *descale_k, const float *descale_v,
+                 void *stream);
+
+/*
+ * attn_hadamard_quant_fp8 -- FP8 input preparation (page "FlashAttention-3 —
+ * 闪电注意力-3", section 3, items 1-3).
+ *   x          [rows, d] bf16 input (any leading shape flattened to rows)
+ *   x8         [rows, d] e4m3 output
+ *   descale    DEVICE pointer to one fp32 output: amax / 448, where amax is
+ *              the largest |value| of the (rotated) tensor
+ *   workspace  DEVICE scratch of attn_hadamard_quant_fp8_workspace_bytes()
+ *              bytes, owned by the caller; its contents on entry do not matter
+ *   signs      DEVICE pointer to d fp32 values, each +1 or -1 (the random
+ *              diagonal), or NULL for no rotation (plain per-tensor FP8)
+ *   d          128 (a power of two the rotation is built for)
+ * With signs != NULL each row is replaced by x diag(signs) H_d / sqrt(d)
+ * (Sylvester Hadamard H_d, computed as a fast Walsh-Hadamard transform in
+ * fp32), which is orthogonal, so (QM)(KM)^T = QK^T.  Then every element is
+ * quantised as E4M3(x * (448/amax)) with round-to-nearest-even and
+ * saturation (fp32 arithmetic).
+ */
+int attn_hadamard_quant_fp8(const void *x, void *x8, float *descale, void *workspace,
+                            long long rows, int d, const float *signs, void *stream);
+
+/* Bytes of device workspace attn_hadamard_quant_fp8 needs. */
+long long attn_hadamard_quant_fp8_workspace_bytes(void);
+
+/*
+ * attn_get_last_device_error -- synchronises `stream`, then reads and clears
+ * the device error word of the current device.  Returns ATTN_OK,
+ * ATTN_ERR_DEVICE_TIMEOUT (a bounded wait ran out inside a kernel) or
+ * ATTN_ERR_CUDA (the synchronisation itself failed).  If `detail` is not
+ * NULL it receives the raw word: bit 0 timeout, bits 8..15 the wait site,
+ * bits 16..31 the low bits of the block index.
+ */
+int attn_get_last_device_error(void *stream, unsigned int *detail);
+
+/* Human-readable name of a status code (static storage). */
+const char *attn_status_string(int status);
+
+/*
+ * Causal tile plan (host and device share this logic; exported for tests).
+ * For the query rows [row0, row1) of one query tile, against Nk keys cut
+ * into tiles of bn keys:
+ *   attn_kv_tile_count  number of leading key tiles that hold at least one
+ *                       visible (row, key) pair (key tiles after that are
+ *                       skipped entirely; 0 if the rows see no key);
+ *   attn_tile_kind      0 = skip (no visible pair), 1 = full (every pair
+ *                       visible: no mask needed), 2 = partial (mask per
+ *                       element), for key tile kt.
+ * row1 is clipped to Nq.  Returns -1 on invalid arguments.
+ */
+int attn_kv_tile_count(int row0, int row1, int Nq, int Nk, int bn, int causal);
+int attn_tile_kind(int row0, int row1, int kt, int Nq, int Nk, int bn, int causal);
+
+/*
+ * Debug hook for the failure path: launches one block that waits, with the
+ * given limit in nanoseconds, on a device barrier nothing ever completes, so
+ * the bounded wait runs out and records ATTN_ERR_DEVICE_TIMEOUT in the
+ * device error word.  Used by the tests to show that a wait that cannot
+ * finish ends with an error status and leaves the context usable.
+ */
+int attn_debug_unsatisfied_wait(long long limit_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBATTN_ATTN_H_ */

@@ -1,0 +1,91 @@
+"""CPU checks of the C boundary: the library loads, exports every symbol that
+include/attn.h declares, and rejects bad arguments with the documented status
+before touching the GPU (no compute calls are made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_140_b200 as ea
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED = 0, 1, 2, 3
+FAKE = 1 << 20  # 16-byte aligned non-null fake device address; never dereferenced
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|long long|char\s*\*|const char\s*\*)\s*\*?\s*(attn_\w+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def test_header_declarations_are_exported():
+    names = declared_functions()
+    assert set(names) == set(ea.EXPORTS), names
+    lib = ctypes.CDLL(ea.lib_path)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    assert ea.attn_status_string(0) == "ok"
+    for s in range(1, 6):
+        assert ea.attn_status_string(s) and ea.attn_status_string(s) != "unknown status"
+    assert ea.attn_status_string(99) == "unknown status"
+
+
+def call(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=1, Nq=128, Nk=128, d=128, causal=0,
+                scale=0.125, dtype=0)
+    args.update(kw)
+    return ea.attn_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["Hq"],
+                       args["Hkv"], args["Nq"], args["Nk"], args["d"], args["causal"], args["scale"],
+                       args["dtype"], stream=0, raise_on_error=False)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), INVALID), (dict(Nq=-3), INVALID), (dict(Nk=-1), INVALID), (dict(Hq=3, Hkv=2), INVALID),
+    (dict(Hkv=0), INVALID), (dict(causal=2), INVALID), (dict(scale=float("nan")), INVALID),
+    (dict(scale=float("inf")), INVALID), (dict(o=0), INVALID), (dict(q=0), INVALID), (dict(dtype=7), INVALID),
+    (dict(d=96), UNSUPPORTED), (dict(d=32), UNSUPPORTED), (dict(d=512), UNSUPPORTED),
+    (dict(dtype=1, d=64), UNSUPPORTED),
+    (dict(q=FAKE + 8), MISALIGNED), (dict(o=FAKE + 2), MISALIGNED), (dict(lse=FAKE + 2), MISALIGNED),
+    (dict(B=0), OK), (dict(Nq=0), OK), (dict(Hq=0), OK),
+])
+def test_argument_errors_before_any_cuda_call(kw, status):
+    assert call(**kw) == status
+
+
+def test_fp8_argument_errors():
+    f = lambda **kw: ea.attn_fwd_fp8(kw.get("q", FAKE), FAKE, FAKE, FAKE, None, 1, 1, 1, 128, 128,
+                                     kw.get("d", 128), 0, 0.1, kw.get("dq", FAKE), FAKE, FAKE, stream=0,
+                                     raise_on_error=False)
+    assert f(d=64) == UNSUPPORTED
+    assert f(dq=0) == INVALID
+    assert f(q=FAKE + 1) == MISALIGNED
+
+
+def test_quant_argument_errors():
+    f = lambda **kw: ea.attn_hadamard_quant_fp8(kw.get("x", FAKE), FAKE, FAKE, kw.get("ws", FAKE),
+                                                kw.get("rows", 4), kw.get("d", 128), kw.get("signs"), stream=0,
+                                                raise_on_error=False)
+    assert f(d=64) == UNSUPPORTED
+    assert f(rows=-1) == INVALID
+    assert f(ws=0) == INVALID
+    assert f(x=FAKE + 4) == MISALIGNED
+    assert f(signs=FAKE + 4) == MISALIGNED
+    assert ea.attn_hadamard_quant_fp8_workspace_bytes() >= 4
+
+
+def test_debug_probe_rejects_bad_limits():
+    assert ea.attn_debug_unsatisfied_wait(0, stream=0, raise_on_error=False) == INVALID
+    assert ea.attn_debug_unsatisfied_wait(10 ** 11, stream=0, raise_on_error=False) == INVALID
+
+
+def test_error_raises():
+    with pytest.raises(ea.AttnError):
+        ea.attn_fwd(FAKE, FAKE, FAKE, FAKE, None, 1, 3, 2, 8, 8, 128, 0, 0.1, 0, stream=0)
