@@ -18,7 +18,7 @@ import os
 __all__ = [
     "ATTN_BF16", "ATTN_FP8_E4M3", "AttnError", "attn_fwd", "attn_fwd_fp8", "attn_hadamard_quant_fp8",
     "attn_hadamard_quant_fp8_workspace_bytes", "attn_get_last_device_error", "attn_status_string",
-    "attn_kv_tile_count", "attn_tile_kind", "attn_debug_unsatisfied_wait", "attention", "lib_path", "EXPORTS",
+    "attn_kv_tile_count", "attn_tile_kind", "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attention", "lib_path", "EXPORTS",
 ]
 
 ATTN_BF16 = 0
@@ -33,7 +33,7 @@ lib_path = os.path.join(_HERE, "libattn.so")
 EXPORTS = (
     "attn_fwd", "attn_fwd_fp8", "attn_hadamard_quant_fp8", "attn_hadamard_quant_fp8_workspace_bytes",
     "attn_get_last_device_error", "attn_status_string", "attn_kv_tile_count", "attn_tile_kind",
-    "attn_debug_unsatisfied_wait",
+    "attn_debug_unsatisfied_wait", "attn_debug_exp2",
 )
 
 if not os.path.exists(lib_path):
@@ -60,6 +60,8 @@ _lib.attn_tile_kind.argtypes = [_I] * 7
 _lib.attn_tile_kind.restype = _I
 _lib.attn_debug_unsatisfied_wait.argtypes = [_LL, _vp]
 _lib.attn_debug_unsatisfied_wait.restype = _I
+_lib.attn_debug_exp2.argtypes = [_vp, _vp, _LL, _I, _vp]
+_lib.attn_debug_exp2.restype = _I
 
 
 class AttnError(RuntimeError):
@@ -137,6 +139,11 @@ def attn_tile_kind(row0, row1, kt, Nq, Nk, bn, causal) -> int:
 def attn_debug_unsatisfied_wait(limit_ns: int, stream=None, raise_on_error=True):
     rc = _lib.attn_debug_unsatisfied_wait(int(limit_ns), _stream(stream))
     return _check(rc, "attn_debug_unsatisfied_wait", raise_on_error)
+
+
+def attn_debug_exp2(x, y, n, mode, stream=None, raise_on_error=True):
+    rc = _lib.attn_debug_exp2(_ptr(x), _ptr(y), int(n), int(mode), _stream(stream))
+    return _check(rc, "attn_debug_exp2", raise_on_error)
 
 
 def attention(q, k, v, causal: bool = False, scale: float | None = None, return_lse: bool = True, stream=None):

@@ -122,6 +122,21 @@ __global__ void unsatisfied_wait_kernel(unsigned int* err, unsigned long long li
   __syncthreads();
 }
 
+__global__ void exp2_probe_kernel(const float* x, float* y, long long n, int mode) {
+  const long long i = 2 * (blockIdx.x * (long long)blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+  float ya, yb;
+  if (mode == 1) {
+    exp2_soft2(a, b, ya, yb);
+  } else {
+    ya = ptx::ex2(a);
+    yb = ptx::ex2(b);
+  }
+  y[i] = ya;
+  if (i + 1 < n) y[i + 1] = yb;
+}
+
 template <class Cfg>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
                int Nk, float scale, const float* dq, const float* dk, const float* dv, DeviceState* st,
@@ -161,15 +176,37 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, int BN, int NQT, int KST, int VST, bool FP8>
+template <int D, int BN, int NQT, int KST, int VST, bool FP8, int EMU>
 int launch_causal(bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                   int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
                   DeviceState* st, cudaStream_t s) {
   if (causal)
-    return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, true, FP8>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk,
-                                                                dv, st, s);
-  return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, false, FP8>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk,
-                                                               dv, st, s);
+    return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq,
+                                                                     dk, dv, st, s);
+  return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq,
+                                                                    dk, dv, st, s);
+}
+
+// Share of softmax exponentials computed in software (out of 8 element pairs);
+// ATTN_EMU overrides the built-in choice for tuning runs.
+int emu_setting(int dflt) {
+  static int v = [] {
+    const char* e = std::getenv("ATTN_EMU");
+    return e == nullptr ? -1 : std::atoi(e);
+  }();
+  return v < 0 ? dflt : v;
+}
+
+template <int D, int BN, int NQT, int KST, int VST, bool FP8>
+int launch_emu(int emu, bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B,
+               int Hq, int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
+               DeviceState* st, cudaStream_t s) {
+  switch (emu) {
+    case 0: return launch_causal<D, BN, NQT, KST, VST, FP8, 0>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
+    case 2: return launch_causal<D, BN, NQT, KST, VST, FP8, 2>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
+    case 4: return launch_causal<D, BN, NQT, KST, VST, FP8, 4>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
+    default: return launch_causal<D, BN, NQT, KST, VST, FP8, 3>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
+  }
 }
 
 int check_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
@@ -250,12 +287,12 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
   const bool c = causal != 0;
   switch (d) {
-    case 64: return launch_causal<64, 128, 2, 3, 3, false>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
-                                                          nullptr, nullptr, st, s);
-    case 128: return launch_causal<128, 128, 2, 2, 2, false>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
-                                                            nullptr, nullptr, st, s);
-    default: return launch_causal<256, 64, 1, 2, 2, false>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
-                                                          nullptr, nullptr, st, s);
+    case 64: return launch_emu<64, 128, 2, 3, 3, false>(emu_setting(3), c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk,
+                                                       scale, nullptr, nullptr, nullptr, st, s);
+    case 128: return launch_emu<128, 128, 2, 2, 2, false>(emu_setting(2), c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk,
+                                                         scale, nullptr, nullptr, nullptr, st, s);
+    default: return launch_causal<256, 64, 1, 2, 2, false, 0>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
+                                                             nullptr, nullptr, st, s);
   }
 }
 
@@ -272,8 +309,8 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float*
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
-  return launch_causal<128, 128, 2, 3, 3, true>(causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, scale, descale_q,
-                                                descale_k, descale_v, st, s);
+  return launch_emu<128, 128, 2, 3, 3, true>(emu_setting(3), causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk,
+                                             scale, descale_q, descale_k, descale_v, st, s);
 }
 
 long long attn_hadamard_quant_fp8_workspace_bytes(void) { return 256; }
@@ -313,6 +350,17 @@ int attn_get_last_device_error(void* stream, unsigned int* detail) {
     return ATTN_ERR_CUDA;
   if (detail != nullptr) *detail = word;
   return word != 0 ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
+}
+
+int attn_debug_exp2(const float* x, float* y, long long n, int mode, void* stream) {
+  if (n < 0 || (mode != 0 && mode != 1) || (n > 0 && (x == nullptr || y == nullptr))) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  int dev = 0, rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
+  const long long pairs = (n + 1) / 2;
+  exp2_probe_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, mode);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int attn_debug_unsatisfied_wait(long long limit_ns, void* stream) {

@@ -15,7 +15,9 @@
 //                       KST / VST-stage shared-memory rings (section 2: the
 //                       next block is fetched while the current one computes);
 //   warp 4*NQT+1        MMA issuer: one thread issues every tcgen05.mma;
-//                       also allocates and frees tensor memory.
+//                       also allocates and frees tensor memory;
+//   warps 4*NQT+2, +3   idle (they complete the control warpgroup, whose
+//                       registers are handed to the softmax warpgroups).
 //
 // Tensor memory (128 lanes x 512 fp32 columns): per query tile t, SB score
 // buffers S of BN columns (P overwrites S in place: BN/2 columns of packed
@@ -41,6 +43,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "exp2_soft.cuh"
 #include "ptx.cuh"
 #include "tiles.h"
 
@@ -62,9 +65,11 @@ struct FwdParams {
 
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
 
-template <int D_, int BN_, int NQT_, int KST_, int VST_, bool CAUSAL_, bool FP8_>
+template <int D_, int BN_, int NQT_, int KST_, int VST_, bool CAUSAL_, bool FP8_, int EMU_ = 0>
 struct FwdCfg {
   static constexpr int D = D_, BN = BN_, NQT = NQT_, KST = KST_, VST = VST_;
+  // software exp2 share on full tiles: element pairs with (pair % 8) < EMU
+  static constexpr int EMU = EMU_;
   static constexpr bool CAUSAL = CAUSAL_, FP8 = FP8_;
   static constexpr int BM = 128;
   static constexpr int SB = NQT == 1 ? 2 : 1;
@@ -105,11 +110,21 @@ struct FwdCfg {
   static constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
   static constexpr uint32_t SMEM_BYTES = OFF_ABORT + 4 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per block");
-  // warps
+  // warps: softmax warpgroups, then one warpgroup holding the TMA warp, the
+  // MMA warp and two idle warps (a whole warpgroup, so that registers can be
+  // moved to the softmax warpgroups with setmaxnreg)
   static constexpr int SM_WARPS = 4 * NQT;
   static constexpr int TMA_WARP = SM_WARPS;
   static constexpr int MMA_WARP = SM_WARPS + 1;
-  static constexpr int NTHREADS = 32 * (SM_WARPS + 2);
+  static constexpr int NTHREADS = 32 * (SM_WARPS + 4);
+  // register split (NQT = 2: 384 threads launch with 168 registers each =
+  // 64512; softmax warpgroups get 224, the control warpgroup keeps 56:
+  // 2*128*224 + 128*56 = 64512)
+  static constexpr int REG_LAUNCH = 65536 / NTHREADS >= 255 ? 255 : (65536 / NTHREADS) / 8 * 8;
+  static constexpr bool SPLIT_REGS = false;
+  static constexpr int REG_SOFTMAX = 232, REG_CONTROL = 40;
+  static_assert(!SPLIT_REGS || 2 * 128 * REG_SOFTMAX + 128 * REG_CONTROL <= NTHREADS * REG_LAUNCH,
+                "register split exceeds the launch allocation");
   static constexpr uint32_t IDESC_QK = ptx::idesc<FP8>(128, BN, false);
   static constexpr uint32_t IDESC_PV = ptx::idesc<FP8>(128, D, true);
 };
@@ -208,6 +223,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
 
   if (warp < Cfg::SM_WARPS) {
     // ------------------------------------------------------------ softmax
+    if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_inc<Cfg::REG_SOFTMAX>();
     const int t = warp >> 2, wq = warp & 3;
     const int row0 = q0 + t * BM;
     const int row = row0 + wq * 32 + lane;
@@ -226,42 +242,41 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       const uint32_t s_taddr = tmem + lane_off + (uint32_t)(si * BN);
-      uint32_t sr[BN];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
-        ptx::tmem_ld32(s_taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
-      ptx::tmem_wait_ld();
-      float s[BN];
-#pragma unroll
-      for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(sr[c]);
       const bool partial = tile_kind(row0, row0 + BM, j, p.Nq, p.Nk, BN, Cfg::CAUSAL) == kTilePartial;
+      const int nvis = (int)(vend - (long long)j * BN);  // visible keys of this tile (masks partial tiles)
+      // ---- pass 1: row max of the (masked) scaled scores
       float m_blk;
-      if (partial) {
-        const long long k0 = (long long)j * BN;
-        float mx = -INFINITY;
+      {
+        uint32_t sr[BN];
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const float x = (k0 + c < vend) ? s[c] * sl2 : -INFINITY;
-          s[c] = x;
-          mx = fmaxf(mx, x);
-        }
-        m_blk = mx;
-      } else {
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        for (int c = 0; c < BN / 32; ++c)
+          ptx::tmem_ld32(s_taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
 #pragma unroll
-        for (int c = 4; c < BN; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
-        }
-        float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-        if (sl2 < 0.f) {  // a negative scale turns the row max into the row min
-          mx = s[0];
+        for (int c = 0; c < BN / 32; ++c) ptx::tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+        if (partial) {
+          float mx = -INFINITY;
 #pragma unroll
-          for (int c = 1; c < BN; ++c) mx = fminf(mx, s[c]);
+          for (int c = 0; c < BN; ++c) mx = fmaxf(mx, (c < nvis) ? __uint_as_float(sr[c]) * sl2 : -INFINITY);
+          m_blk = mx;
+        } else if (sl2 >= 0.f) {
+          float a0 = __uint_as_float(sr[0]), a1 = __uint_as_float(sr[1]);
+          float a2 = __uint_as_float(sr[2]), a3 = __uint_as_float(sr[3]);
+#pragma unroll
+          for (int c = 4; c < BN; c += 8) {
+            a0 = ptx::fmax3(a0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+            a1 = ptx::fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+            if (c + 4 < BN) {
+              a2 = ptx::fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+              a3 = ptx::fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+            }
+          }
+          m_blk = ptx::fmax3(a0, a1, fmaxf(a2, a3)) * sl2;
+        } else {  // a negative scale turns the row max into the row min
+          float mn = __uint_as_float(sr[0]);
+#pragma unroll
+          for (int c = 1; c < BN; ++c) mn = fminf(mn, __uint_as_float(sr[c]));
+          m_blk = mn * sl2;
         }
-        m_blk = mx * sl2;
       }
       float alpha = 1.f;
       bool resc = false;
@@ -272,34 +287,63 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         l *= alpha;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // exponentiate, accumulate the row sum and pack P in one pass, so each
-      // score register dies as soon as its packed weight exists
-      float l0 = 0.f, l1 = 0.f;
-      uint32_t pk[Cfg::P_COLS];
-      constexpr int PER = Cfg::FP8 ? 4 : 2;  // weights per 32-bit TMEM column
+      // ---- pass 2: 32-column chunks re-read from TMEM (the next chunk's load
+      // is in flight while this one is exponentiated); P is packed and stored
+      // over the columns already consumed
+      uint64_t lsum = ptx::f2(0.f, 0.f);
+      const uint64_t sl2x2 = ptx::f2(sl2, sl2), negm2 = ptx::f2(-m_use, -m_use);
+      constexpr int NCHK = BN / 32;
+      constexpr int PW = Cfg::FP8 ? 8 : 16;  // packed P words per 32 scores
+      uint32_t buf[2][32];
+      ptx::tmem_ld32(s_taddr, buf[0]);
+      ptx::tmem_wait_ld_dep(buf[0]);
 #pragma unroll
-      for (int c = 0; c < Cfg::P_COLS; ++c) {
-        float e[PER];
+      for (int ch = 0; ch < NCHK; ++ch) {
+        uint32_t(&cur)[32] = buf[ch & 1];
+        if (ch + 1 < NCHK) ptx::tmem_ld32(s_taddr + 32 * (ch + 1), buf[(ch + 1) & 1]);
+        uint32_t pk[PW];
 #pragma unroll
-        for (int u = 0; u < PER; ++u) {
-          const float x = s[PER * c + u];
-          e[u] = ptx::ex2(partial ? (x - m_use) : fmaf(x, sl2, -m_use));
+        for (int c = 0; c < 16; ++c) {
+          const float s0 = __uint_as_float(cur[2 * c]), s1 = __uint_as_float(cur[2 * c + 1]);
+          float e0, e1;
+          if (partial) {
+            const int col = 32 * ch + 2 * c;
+            e0 = ptx::ex2((col < nvis ? s0 * sl2 : -INFINITY) - m_use);
+            e1 = ptx::ex2((col + 1 < nvis ? s1 * sl2 : -INFINITY) - m_use);
+          } else {
+            const uint64_t x = ptx::ffma2(ptx::f2(s0, s1), sl2x2, negm2);
+            float x0, x1;
+            ptx::unf2(x, x0, x1);
+            if (((16 * ch + c) % 8) < Cfg::EMU) {
+              exp2_soft2(x0, x1, e0, e1);
+            } else {
+              e0 = ptx::ex2(x0);
+              e1 = ptx::ex2(x1);
+            }
+          }
+          lsum = ptx::fadd2(lsum, ptx::f2(e0, e1));
+          if constexpr (Cfg::FP8) {
+            if (c % 2 == 0) {
+              cur[2 * c] = __float_as_uint(e0);  // held for the 4-wide e4m3 pack
+              cur[2 * c + 1] = __float_as_uint(e1);
+            } else {
+              pk[c / 2] = ptx::pack_e4m3x4(__uint_as_float(cur[2 * c - 2]), __uint_as_float(cur[2 * c - 1]), e0, e1);
+            }
+          } else {
+            pk[c] = ptx::pack_bf16x2(e0, e1);
+          }
         }
-        if constexpr (Cfg::FP8) {
-          l0 += e[0] + e[1];
-          l1 += e[2] + e[3];
-          pk[c] = ptx::pack_e4m3x4(e[0], e[1], e[2], e[3]);
-        } else {
-          l0 += e[0];
-          l1 += e[1];
-          pk[c] = ptx::pack_bf16x2(e[0], e[1]);
-        }
+        if constexpr (Cfg::FP8)
+          ptx::tmem_st8(s_taddr + (uint32_t)(PW * ch), pk);
+        else
+          ptx::tmem_st16(s_taddr + (uint32_t)(PW * ch), pk);
+        if (ch + 1 < NCHK) ptx::tmem_wait_ld_dep(buf[(ch + 1) & 1]);
       }
-      l += l0 + l1;
-#pragma unroll
-      for (int c = 0; c < Cfg::P_COLS / 32; ++c)
-        ptx::tmem_st32(s_taddr + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * c]));
-      if constexpr (Cfg::P_COLS % 32 == 16) ptx::tmem_st16(s_taddr + (Cfg::P_COLS / 32) * 32, &pk[Cfg::P_COLS - 16]);
+      {
+        float la, lb;
+        ptx::unf2(lsum, la, lb);
+        l += la + lb;
+      }
       ptx::tmem_wait_st();
       if (j > 0) {
         // PV(t, j-1) must be complete before P(t, j) is released (and before
@@ -317,7 +361,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
           ptx::tmem_ld32(o_taddr + 32 * c, r);
-          ptx::tmem_wait_ld();
+          ptx::tmem_wait_ld_dep(r);
 #pragma unroll
           for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * a);
           ptx::tmem_st32(o_taddr + 32 * c, r);
@@ -344,7 +388,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         uint32_t r[32];
         if (nt > 0) {
           ptx::tmem_ld32(o_taddr + 32 * c, r);
-          ptx::tmem_wait_ld();
+          ptx::tmem_wait_ld_dep(r);
         }
         uint32_t w[16];
 #pragma unroll
@@ -364,6 +408,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
     }
   } else if (warp == Cfg::TMA_WARP) {
     // ------------------------------------------------------------ producer
+    if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_dec<Cfg::REG_CONTROL>();
     if (lane == 0) {
       int k_issued[KST], v_issued[VST];
 #pragma unroll
@@ -421,6 +466,9 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         if (v_issued[s] > 0) wait_bar(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
     }
   } else {
+    if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_dec<Cfg::REG_CONTROL>();
+  }
+  if (warp == Cfg::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = true;

@@ -158,6 +158,14 @@ int attn_tile_kind(int row0, int row1, int kt, int Nq, int Nk, int bn, int causa
  */
 int attn_debug_unsatisfied_wait(long long limit_ns, void *stream);
 
+/*
+ * Debug hook for the softmax exponential: y[i] = 2^x[i] for n values, as the
+ * attention kernel computes it: mode 0 the hardware approximation
+ * (ex2.approx), mode 1 the software polynomial (page "FlashAttention-4震撼发布",
+ * software emulation of the exponential).  x and y are device pointers.
+ */
+int attn_debug_exp2(const float *x, float *y, long long n, int mode, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
