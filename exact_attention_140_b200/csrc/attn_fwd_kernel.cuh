@@ -42,6 +42,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "exp2_soft.cuh"
 #include "ptx.cuh"
@@ -121,8 +122,8 @@ struct FwdCfg {
   // 64512; softmax warpgroups get 224, the control warpgroup keeps 56:
   // 2*128*224 + 128*56 = 64512)
   static constexpr int REG_LAUNCH = 65536 / NTHREADS >= 255 ? 255 : (65536 / NTHREADS) / 8 * 8;
-  static constexpr bool SPLIT_REGS = false;
-  static constexpr int REG_SOFTMAX = 232, REG_CONTROL = 40;
+  static constexpr bool SPLIT_REGS = NQT == 2;
+  static constexpr int REG_SOFTMAX = 200, REG_CONTROL = 104;
   static_assert(!SPLIT_REGS || 2 * 128 * REG_SOFTMAX + 128 * REG_CONTROL <= NTHREADS * REG_LAUNCH,
                 "register split exceeds the launch allocation");
   static constexpr uint32_t IDESC_QK = ptx::idesc<FP8>(128, BN, false);
@@ -144,8 +145,12 @@ struct WaitCtx {
 // Bounded mbarrier wait: true when the phase with `parity` has completed;
 // false after the time limit (recording the site in the error word and
 // raising the block's abort flag) or when another role already aborted.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, const WaitCtx& c, uint32_t site) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+// The first probe is inline; only a wait that does not succeed at once pays
+// for the call into the polling loop.  The polling loop is instantiated once
+// per warp role (ROLE), because roles run under different register budgets
+// (setmaxnreg) and a called function is compiled for one budget.
+template <int ROLE>
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, const WaitCtx& c, uint32_t site) {
   const uint64_t t0 = ptx::globaltimer();
   for (;;) {
 #pragma unroll 1
@@ -160,6 +165,12 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, const WaitC
     }
   }
 }
+template <int ROLE = 0>
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const WaitCtx& c, uint32_t site) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  return wait_bar_slow<ROLE>(bar, parity, c, site);
+}
+enum : int { kRoleSoftmax = 0, kRoleProducer = 1, kRoleMma = 2 };
 
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
@@ -237,46 +248,44 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int si = t * SB + (j % SB);
-      ok = wait_bar(bar(Cfg::B_SFULL + si), (uint32_t)((j / SB) & 1), wc, kSiteSFull);
+      ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_SFULL + si), (uint32_t)((j / SB) & 1), wc, kSiteSFull);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
       const uint32_t s_taddr = tmem + lane_off + (uint32_t)(si * BN);
       const bool partial = tile_kind(row0, row0 + BM, j, p.Nq, p.Nk, BN, Cfg::CAUSAL) == kTilePartial;
       const int nvis = (int)(vend - (long long)j * BN);  // visible keys of this tile (masks partial tiles)
-      // ---- pass 1: row max of the (masked) scaled scores
+      // ---- one read of the whole score row (one TMEM load latency per tile)
+      uint32_t sr[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c)
+        ptx::tmem_ld32(s_taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) ptx::tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
       float m_blk;
-      {
-        uint32_t sr[BN];
+      if (partial) {
+        float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
-          ptx::tmem_ld32(s_taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, (c < nvis) ? __uint_as_float(sr[c]) * sl2 : -INFINITY);
+        m_blk = mx;
+      } else if (sl2 >= 0.f) {
+        float a0 = __uint_as_float(sr[0]), a1 = __uint_as_float(sr[1]);
+        float a2 = __uint_as_float(sr[2]), a3 = __uint_as_float(sr[3]);
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) ptx::tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
-        if (partial) {
-          float mx = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < BN; ++c) mx = fmaxf(mx, (c < nvis) ? __uint_as_float(sr[c]) * sl2 : -INFINITY);
-          m_blk = mx;
-        } else if (sl2 >= 0.f) {
-          float a0 = __uint_as_float(sr[0]), a1 = __uint_as_float(sr[1]);
-          float a2 = __uint_as_float(sr[2]), a3 = __uint_as_float(sr[3]);
-#pragma unroll
-          for (int c = 4; c < BN; c += 8) {
-            a0 = ptx::fmax3(a0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-            a1 = ptx::fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-            if (c + 4 < BN) {
-              a2 = ptx::fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-              a3 = ptx::fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
-            }
+        for (int c = 4; c < BN; c += 8) {
+          a0 = ptx::fmax3(a0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+          a1 = ptx::fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+          if (c + 4 < BN) {
+            a2 = ptx::fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+            a3 = ptx::fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
           }
-          m_blk = ptx::fmax3(a0, a1, fmaxf(a2, a3)) * sl2;
-        } else {  // a negative scale turns the row max into the row min
-          float mn = __uint_as_float(sr[0]);
-#pragma unroll
-          for (int c = 1; c < BN; ++c) mn = fminf(mn, __uint_as_float(sr[c]));
-          m_blk = mn * sl2;
         }
+        m_blk = ptx::fmax3(a0, a1, fmaxf(a2, a3)) * sl2;
+      } else {  // a negative scale turns the row max into the row min
+        float mn = __uint_as_float(sr[0]);
+#pragma unroll
+        for (int c = 1; c < BN; ++c) mn = fminf(mn, __uint_as_float(sr[c]));
+        m_blk = mn * sl2;
       }
       float alpha = 1.f;
       bool resc = false;
@@ -287,61 +296,66 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         l *= alpha;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // ---- pass 2: 32-column chunks re-read from TMEM (the next chunk's load
-      // is in flight while this one is exponentiated); P is packed and stored
-      // over the columns already consumed
-      uint64_t lsum = ptx::f2(0.f, 0.f);
+      // ---- exponentiate 32 columns at a time; each chunk's packed P is
+      // stored at once (over score columns already read), so the registers of
+      // a chunk die before the next chunk is processed
+      uint64_t lsum[4] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
       const uint64_t sl2x2 = ptx::f2(sl2, sl2), negm2 = ptx::f2(-m_use, -m_use);
-      constexpr int NCHK = BN / 32;
       constexpr int PW = Cfg::FP8 ? 8 : 16;  // packed P words per 32 scores
-      uint32_t buf[2][32];
-      ptx::tmem_ld32(s_taddr, buf[0]);
-      ptx::tmem_wait_ld_dep(buf[0]);
+      // The tile kind is resolved once, outside the unrolled loop: one loop
+      // body per kind, no per-element branches.
+      auto exp_row = [&](auto partial_tag) {
+        constexpr bool PARTIAL = decltype(partial_tag)::value;
 #pragma unroll
-      for (int ch = 0; ch < NCHK; ++ch) {
-        uint32_t(&cur)[32] = buf[ch & 1];
-        if (ch + 1 < NCHK) ptx::tmem_ld32(s_taddr + 32 * (ch + 1), buf[(ch + 1) & 1]);
-        uint32_t pk[PW];
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          uint32_t pk[PW];
+          [[maybe_unused]] float hold0 = 0.f, hold1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float s0 = __uint_as_float(cur[2 * c]), s1 = __uint_as_float(cur[2 * c + 1]);
-          float e0, e1;
-          if (partial) {
+          for (int c = 0; c < 16; ++c) {
             const int col = 32 * ch + 2 * c;
-            e0 = ptx::ex2((col < nvis ? s0 * sl2 : -INFINITY) - m_use);
-            e1 = ptx::ex2((col + 1 < nvis ? s1 * sl2 : -INFINITY) - m_use);
-          } else {
-            const uint64_t x = ptx::ffma2(ptx::f2(s0, s1), sl2x2, negm2);
-            float x0, x1;
-            ptx::unf2(x, x0, x1);
-            if (((16 * ch + c) % 8) < Cfg::EMU) {
-              exp2_soft2(x0, x1, e0, e1);
+            const float s0 = __uint_as_float(sr[col]), s1 = __uint_as_float(sr[col + 1]);
+            float e0, e1;
+            if constexpr (PARTIAL) {
+              e0 = ptx::ex2((col < nvis ? s0 * sl2 : -INFINITY) - m_use);
+              e1 = ptx::ex2((col + 1 < nvis ? s1 * sl2 : -INFINITY) - m_use);
             } else {
-              e0 = ptx::ex2(x0);
-              e1 = ptx::ex2(x1);
+              const uint64_t x = ptx::ffma2(ptx::f2(s0, s1), sl2x2, negm2);
+              float x0, x1;
+              ptx::unf2(x, x0, x1);
+              if constexpr (true) {
+                if (((16 * ch + c) % 8) < Cfg::EMU) {
+                  exp2_soft2(x0, x1, e0, e1);
+                } else {
+                  e0 = ptx::ex2(x0);
+                  e1 = ptx::ex2(x1);
+                }
+              }
+            }
+            lsum[c % 4] = ptx::fadd2(lsum[c % 4], ptx::f2(e0, e1));
+            if constexpr (Cfg::FP8) {
+              if (c % 2 == 0) {
+                hold0 = e0;
+                hold1 = e1;
+              } else {
+                pk[c / 2] = ptx::pack_e4m3x4(hold0, hold1, e0, e1);
+              }
+            } else {
+              pk[c] = ptx::pack_bf16x2(e0, e1);
             }
           }
-          lsum = ptx::fadd2(lsum, ptx::f2(e0, e1));
-          if constexpr (Cfg::FP8) {
-            if (c % 2 == 0) {
-              cur[2 * c] = __float_as_uint(e0);  // held for the 4-wide e4m3 pack
-              cur[2 * c + 1] = __float_as_uint(e1);
-            } else {
-              pk[c / 2] = ptx::pack_e4m3x4(__uint_as_float(cur[2 * c - 2]), __uint_as_float(cur[2 * c - 1]), e0, e1);
-            }
-          } else {
-            pk[c] = ptx::pack_bf16x2(e0, e1);
-          }
+          if constexpr (Cfg::FP8)
+            ptx::tmem_st8(s_taddr + (uint32_t)(PW * ch), pk);
+          else
+            ptx::tmem_st16(s_taddr + (uint32_t)(PW * ch), pk);
         }
-        if constexpr (Cfg::FP8)
-          ptx::tmem_st8(s_taddr + (uint32_t)(PW * ch), pk);
-        else
-          ptx::tmem_st16(s_taddr + (uint32_t)(PW * ch), pk);
-        if (ch + 1 < NCHK) ptx::tmem_wait_ld_dep(buf[(ch + 1) & 1]);
-      }
+      };
+      if (partial)
+        exp_row(std::true_type{});
+      else
+        exp_row(std::false_type{});
       {
         float la, lb;
-        ptx::unf2(lsum, la, lb);
+        ptx::unf2(ptx::fadd2(ptx::fadd2(lsum[0], lsum[1]), ptx::fadd2(lsum[2], lsum[3])), la, lb);
         l += la + lb;
       }
       ptx::tmem_wait_st();
@@ -350,7 +364,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         // O_t is rescaled).  Observing every o_done phase in order keeps the
         // barrier within one phase of this thread's view, so parity waits are
         // unambiguous.
-        ok = wait_bar(bar(Cfg::B_ODONE + t), (uint32_t)((j - 1) & 1), wc, kSiteODone);
+        ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_ODONE + t), (uint32_t)((j - 1) & 1), wc, kSiteODone);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
       }
@@ -373,7 +387,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
     }
     // ------------------------------------------------------------ epilogue
     if (ok && nt > 0) {
-      ok = wait_bar(bar(Cfg::B_ODONE + t), (uint32_t)((nt - 1) & 1), wc, kSiteODone);
+      ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_ODONE + t), (uint32_t)((nt - 1) & 1), wc, kSiteODone);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
@@ -429,7 +443,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       }
       for (int j = 0; j < nmax; ++j) {
         const int ks = j % KST;
-        if (j >= KST && !wait_bar(bar(Cfg::B_KEMPTY + ks), (uint32_t)(((j / KST) - 1) & 1), wc, kSiteKEmpty))
+        if (j >= KST && !wait_bar<kRoleProducer>(bar(Cfg::B_KEMPTY + ks), (uint32_t)(((j / KST) - 1) & 1), wc, kSiteKEmpty))
           break;
         {
           const uint32_t fb = bar(Cfg::B_KFULL + ks);
@@ -441,7 +455,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
           ++k_issued[ks];
         }
         const int vs = j % VST;
-        if (j >= VST && !wait_bar(bar(Cfg::B_VEMPTY + vs), (uint32_t)(((j / VST) - 1) & 1), wc, kSiteVEmpty))
+        if (j >= VST && !wait_bar<kRoleProducer>(bar(Cfg::B_VEMPTY + vs), (uint32_t)(((j / VST) - 1) & 1), wc, kSiteVEmpty))
           break;
         {
           const uint32_t fb = bar(Cfg::B_VFULL + vs);
@@ -457,13 +471,13 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       // normal path, where the consumers have already seen them all).
 #pragma unroll
       for (int t = 0; t < NQT; ++t)
-        if (q_issued[t]) wait_bar(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
+        if (q_issued[t]) wait_bar<kRoleProducer>(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
 #pragma unroll
       for (int s = 0; s < KST; ++s)
-        if (k_issued[s] > 0) wait_bar(bar(Cfg::B_KFULL + s), (uint32_t)((k_issued[s] - 1) & 1), wc, kSiteKFull);
+        if (k_issued[s] > 0) wait_bar<kRoleProducer>(bar(Cfg::B_KFULL + s), (uint32_t)((k_issued[s] - 1) & 1), wc, kSiteKFull);
 #pragma unroll
       for (int s = 0; s < VST; ++s)
-        if (v_issued[s] > 0) wait_bar(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
+        if (v_issued[s] > 0) wait_bar<kRoleProducer>(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
     }
   } else {
     if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_dec<Cfg::REG_CONTROL>();
@@ -474,17 +488,17 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       bool ok = true;
 #pragma unroll
       for (int t = 0; t < NQT && ok; ++t)
-        if (n_kv[t] > 0) ok = wait_bar(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
+        if (n_kv[t] > 0) ok = wait_bar<kRoleMma>(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
       ptx::tc_fence_after();
       const uint32_t q_s = sbase + Cfg::OFF_Q, k_s = sbase + Cfg::OFF_K, v_s = sbase + Cfg::OFF_V;
       for (int j = 0; ok && j <= nmax; ++j) {
         const bool has_k = j < nmax, has_v = j >= 1;
         if (has_k) {
-          ok = wait_bar(bar(Cfg::B_KFULL + j % KST), (uint32_t)((j / KST) & 1), wc, kSiteKFull);
+          ok = wait_bar<kRoleMma>(bar(Cfg::B_KFULL + j % KST), (uint32_t)((j / KST) & 1), wc, kSiteKFull);
           if (!ok) break;
         }
         if (has_v) {
-          ok = wait_bar(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc, kSiteVFull);
+          ok = wait_bar<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc, kSiteVFull);
           if (!ok) break;
         }
         ptx::tc_fence_after();
@@ -493,14 +507,15 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
           auto issue_qk = [&]() {
             if (!(has_k && j < n_kv[t])) return;
             const uint32_t d_t = tmem + (uint32_t)((t * SB + j % SB) * BN);
-            const uint32_t qa = q_s + t * Cfg::QT_BYTES;
-            const uint32_t kb = k_s + (j % KST) * Cfg::KV_BYTES;
+            // descriptors advance by 32 bytes (>> 4 = 2) per K step inside a
+            // 128-byte chunk and by one chunk (CH_Q / CH_KV bytes) after four
+            const uint64_t ad0 = ptx::sdesc_sw128(q_s + t * Cfg::QT_BYTES, 16u, 1024u);
+            const uint64_t bd0 = ptx::sdesc_sw128(k_s + (j % KST) * Cfg::KV_BYTES, 16u, 1024u);
 #pragma unroll
             for (int kk = 0; kk < Cfg::QK_STEPS; ++kk) {
-              const uint32_t off = (uint32_t)kk * 32u;  // bytes along the reduction dim
-              const uint32_t ch = off / 128u, in = off % 128u;
-              const uint64_t ad = ptx::sdesc_sw128(qa + ch * Cfg::CH_Q + in, 16u, 1024u);
-              const uint64_t bd = ptx::sdesc_sw128(kb + ch * Cfg::CH_KV + in, 16u, 1024u);
+              const uint32_t ch = (uint32_t)kk / 4u, in = (uint32_t)kk % 4u;
+              const uint64_t ad = ad0 + (uint64_t)((ch * Cfg::CH_Q + in * 32u) >> 4);
+              const uint64_t bd = bd0 + (uint64_t)((ch * Cfg::CH_KV + in * 32u) >> 4);
               ptx::mma_ss<Cfg::FP8>(d_t, ad, bd, Cfg::IDESC_QK, kk > 0 ? 1u : 0u);
             }
             ptx::tc_commit(bar(Cfg::B_SFULL + t * SB + j % SB));
@@ -509,16 +524,15 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
             const int jj = j - 1;
             if (!(has_v && jj < n_kv[t])) return true;
             const int si = t * SB + jj % SB;
-            if (!wait_bar(bar(Cfg::B_PFULL + si), (uint32_t)((jj / SB) & 1), wc, kSitePFull)) return false;
+            if (!wait_bar<kRoleMma>(bar(Cfg::B_PFULL + si), (uint32_t)((jj / SB) & 1), wc, kSitePFull)) return false;
             ptx::tc_fence_after();
             const uint32_t d_t = tmem + (uint32_t)(Cfg::O_COL0 + t * D);
             const uint32_t a_t = tmem + (uint32_t)(si * BN);
-            const uint32_t vb = v_s + (jj % VST) * Cfg::KV_BYTES;
+            const uint64_t bd0 = ptx::sdesc_sw128(v_s + (jj % VST) * Cfg::KV_BYTES, Cfg::CH_KV, 1024u);
 #pragma unroll
             for (int kk = 0; kk < Cfg::PV_STEPS; ++kk) {
-              const uint64_t bd = ptx::sdesc_sw128(vb + (uint32_t)kk * Cfg::KSTEP * 128u, Cfg::CH_KV, 1024u);
-              ptx::mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV,
-                                    (jj > 0 || kk > 0) ? 1u : 0u);
+              const uint64_t bd = bd0 + (uint64_t)(((uint32_t)kk * Cfg::KSTEP * 128u) >> 4);
+              ptx::mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
             }
             ptx::tc_commit(bar(Cfg::B_ODONE + t));
             return true;
@@ -538,7 +552,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       }
       // All issued MMAs must finish before tensor memory is freed.
       ptx::tc_commit(bar(Cfg::B_DRAIN));
-      wait_bar(bar(Cfg::B_DRAIN), 0u, wc, kSiteDrain);
+      wait_bar<kRoleMma>(bar(Cfg::B_DRAIN), 0u, wc, kSiteDrain);
     }
   }
 
