@@ -330,7 +330,7 @@ def run_ours(args, cfg, name):
     kern_avg_s = float(np.mean(kern_ms)) * 1e-3
     achieved = f / kern_avg_s / 1e12
     peak = peaks["bf16"] * (2.0 if fp8 else 1.0)
-    traffic = TRAFFIC.get(name)
+    traffic = traffic_bytes(name)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -357,9 +357,29 @@ def run_ours(args, cfg, name):
     return 0
 
 
-# dram bytes (read + write) per launch of the attention kernel from an ncu capture of
-# the same kernel; null until taken for the current kernel
-TRAFFIC: dict = {}
+def kernel_source_hash() -> str:
+    import hashlib
+    csrc = os.path.join(ROOT, "exact_attention_140_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(f.encode())
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_bytes(name):
+    """DRAM bytes per launch from the committed ncu record, or None when the
+    kernel sources changed since it was taken (or the workload has none)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get(name)
 
 
 def main():

@@ -176,15 +176,15 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, int BN, int NQT, int KST, int VST, bool FP8, int EMU>
+template <int D, int BN, int NQT, int KST, int VST, bool FP8, int EMU, int SB = (NQT == 1 ? 2 : 1)>
 int launch_causal(bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                   int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
                   DeviceState* st, cudaStream_t s) {
   if (causal)
-    return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq,
-                                                                     dk, dv, st, s);
-  return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq,
-                                                                    dk, dv, st, s);
+    return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU, SB>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale,
+                                                                         dq, dk, dv, st, s);
+  return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU, SB>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale,
+                                                                        dq, dk, dv, st, s);
 }
 
 // Share of softmax exponentials computed in software (out of 8 element pairs);
@@ -287,10 +287,12 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
   const bool c = causal != 0;
   switch (d) {
-    case 64: return launch_emu<64, 128, 2, 3, 3, false>(emu_setting(3), c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk,
-                                                       scale, nullptr, nullptr, nullptr, st, s);
-    case 128: return launch_emu<128, 128, 2, 2, 2, false>(emu_setting(2), c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk,
-                                                         scale, nullptr, nullptr, nullptr, st, s);
+    case 64:
+      return launch_emu<64, 128, 2, 3, 3, false>(emu_setting(3), c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale,
+                                                 nullptr, nullptr, nullptr, st, s);
+    case 128:
+      return launch_emu<128, 128, 2, 2, 2, false>(emu_setting(2), c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale,
+                                                  nullptr, nullptr, nullptr, st, s);
     default: return launch_causal<256, 64, 1, 2, 2, false, 0>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
                                                              nullptr, nullptr, st, s);
   }

@@ -66,14 +66,16 @@ struct FwdParams {
 
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
 
-template <int D_, int BN_, int NQT_, int KST_, int VST_, bool CAUSAL_, bool FP8_, int EMU_ = 0>
+template <int D_, int BN_, int NQT_, int KST_, int VST_, bool CAUSAL_, bool FP8_, int EMU_ = 0,
+          int SB_ = (NQT_ == 1 ? 2 : 1)>
 struct FwdCfg {
   static constexpr int D = D_, BN = BN_, NQT = NQT_, KST = KST_, VST = VST_;
   // software exp2 share on full tiles: element pairs with (pair % 8) < EMU
   static constexpr int EMU = EMU_;
   static constexpr bool CAUSAL = CAUSAL_, FP8 = FP8_;
   static constexpr int BM = 128;
-  static constexpr int SB = NQT == 1 ? 2 : 1;
+  static constexpr int SB = SB_;  // score buffers per query tile
+  static_assert(SB == 1 || SB == 2, "one or two score buffers");
   static constexpr int ELEM = FP8 ? 1 : 2;
   static constexpr int NCH = D * ELEM / 128;  // 128-byte column chunks per row
   static constexpr int BOXE = 128 / ELEM;     // elements per chunk row
@@ -100,7 +102,8 @@ struct FwdCfg {
   static constexpr int B_SFULL = B_VEMPTY + VST;
   static constexpr int B_PFULL = B_SFULL + NQT * SB;
   static constexpr int B_ODONE = B_PFULL + NQT * SB;
-  static constexpr int B_DRAIN = B_ODONE + NQT;
+  static constexpr int B_OFINAL = B_ODONE + NQT;
+  static constexpr int B_DRAIN = B_OFINAL + NQT;
   static constexpr int NBAR = B_DRAIN + 1;
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr uint32_t OFF_Q = 0;
@@ -213,7 +216,10 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       ptx::mbar_init(bar(Cfg::B_SFULL + i), 1);
       ptx::mbar_init(bar(Cfg::B_PFULL + i), 128);
     }
-    for (int t = 0; t < NQT; ++t) ptx::mbar_init(bar(Cfg::B_ODONE + t), 1);
+    for (int t = 0; t < NQT; ++t) {
+      ptx::mbar_init(bar(Cfg::B_ODONE + t), 1);
+      ptx::mbar_init(bar(Cfg::B_OFINAL + t), 1);
+    }
     ptx::mbar_init(bar(Cfg::B_DRAIN), 1);
     *abort_flag = 0u;
     ptx::fence_mbar_init();
@@ -359,16 +365,15 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         l += la + lb;
       }
       ptx::tmem_wait_st();
-      if (j > 0) {
-        // PV(t, j-1) must be complete before P(t, j) is released (and before
-        // O_t is rescaled).  Observing every o_done phase in order keeps the
-        // barrier within one phase of this thread's view, so parity waits are
-        // unambiguous.
+      if (__any_sync(0xffffffffu, resc)) {
+        // O_t must hold exactly the products of key tiles < j: wait for
+        // PV(t, j-1).  Whenever S(t, j) is ready, PV(t, j-2) has completed (it
+        // was issued before QK(t, j)) and PV(t, j) is not issued yet, so the
+        // o_done barrier has completed j-1 or j phases and the parity test
+        // for phase j-1 is unambiguous.
         ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_ODONE + t), (uint32_t)((j - 1) & 1), wc, kSiteODone);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-      }
-      if (__any_sync(0xffffffffu, resc)) {
         ptx::tc_fence_after();
         const float a = resc ? alpha : 1.f;
 #pragma unroll 1
@@ -386,8 +391,8 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       ptx::mbar_arrive(bar(Cfg::B_PFULL + si));
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && nt > 0) {
-      ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_ODONE + t), (uint32_t)((nt - 1) & 1), wc, kSiteODone);
+    if (ok && nt > 0) {  // o_final completes once, after the tile's last PV
+      ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_OFINAL + t), 0u, wc, kSiteODone);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
@@ -491,64 +496,85 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         if (n_kv[t] > 0) ok = wait_bar<kRoleMma>(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
       ptx::tc_fence_after();
       const uint32_t q_s = sbase + Cfg::OFF_Q, k_s = sbase + Cfg::OFF_K, v_s = sbase + Cfg::OFF_V;
+      auto issue_qk = [&](int t, int j) {
+        const uint32_t d_t = tmem + (uint32_t)((t * SB + j % SB) * BN);
+        // descriptors advance by 32 bytes (>> 4 = 2) per K step inside a
+        // 128-byte chunk and by one chunk (CH_Q / CH_KV bytes) after four
+        const uint64_t ad0 = ptx::sdesc_sw128(q_s + t * Cfg::QT_BYTES, 16u, 1024u);
+        const uint64_t bd0 = ptx::sdesc_sw128(k_s + (j % KST) * Cfg::KV_BYTES, 16u, 1024u);
+#pragma unroll
+        for (int kk = 0; kk < Cfg::QK_STEPS; ++kk) {
+          const uint32_t ch = (uint32_t)kk / 4u, in = (uint32_t)kk % 4u;
+          const uint64_t ad = ad0 + (uint64_t)((ch * Cfg::CH_Q + in * 32u) >> 4);
+          const uint64_t bd = bd0 + (uint64_t)((ch * Cfg::CH_KV + in * 32u) >> 4);
+          ptx::mma_ss<Cfg::FP8>(d_t, ad, bd, Cfg::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        ptx::tc_commit(bar(Cfg::B_SFULL + t * SB + j % SB));
+      };
+      auto issue_pv = [&](int t, int jj) -> bool {
+        const int si = t * SB + jj % SB;
+        if (!wait_bar<kRoleMma>(bar(Cfg::B_PFULL + si), (uint32_t)((jj / SB) & 1), wc, kSitePFull)) return false;
+        ptx::tc_fence_after();
+        const uint32_t d_t = tmem + (uint32_t)(Cfg::O_COL0 + t * D);
+        const uint32_t a_t = tmem + (uint32_t)(si * BN);
+        const uint64_t bd0 = ptx::sdesc_sw128(v_s + (jj % VST) * Cfg::KV_BYTES, Cfg::CH_KV, 1024u);
+#pragma unroll
+        for (int kk = 0; kk < Cfg::PV_STEPS; ++kk) {
+          const uint64_t bd = bd0 + (uint64_t)(((uint32_t)kk * Cfg::KSTEP * 128u) >> 4);
+          ptx::mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::tc_commit(bar(Cfg::B_ODONE + t));
+        if (jj == n_kv[t] - 1) ptx::tc_commit(bar(Cfg::B_OFINAL + t));
+        return true;
+      };
       for (int j = 0; ok && j <= nmax; ++j) {
         const bool has_k = j < nmax, has_v = j >= 1;
-        if (has_k) {
-          ok = wait_bar<kRoleMma>(bar(Cfg::B_KFULL + j % KST), (uint32_t)((j / KST) & 1), wc, kSiteKFull);
-          if (!ok) break;
-        }
-        if (has_v) {
-          ok = wait_bar<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc, kSiteVFull);
-          if (!ok) break;
-        }
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int t = 0; t < NQT; ++t) {
-          auto issue_qk = [&]() {
-            if (!(has_k && j < n_kv[t])) return;
-            const uint32_t d_t = tmem + (uint32_t)((t * SB + j % SB) * BN);
-            // descriptors advance by 32 bytes (>> 4 = 2) per K step inside a
-            // 128-byte chunk and by one chunk (CH_Q / CH_KV bytes) after four
-            const uint64_t ad0 = ptx::sdesc_sw128(q_s + t * Cfg::QT_BYTES, 16u, 1024u);
-            const uint64_t bd0 = ptx::sdesc_sw128(k_s + (j % KST) * Cfg::KV_BYTES, 16u, 1024u);
-#pragma unroll
-            for (int kk = 0; kk < Cfg::QK_STEPS; ++kk) {
-              const uint32_t ch = (uint32_t)kk / 4u, in = (uint32_t)kk % 4u;
-              const uint64_t ad = ad0 + (uint64_t)((ch * Cfg::CH_Q + in * 32u) >> 4);
-              const uint64_t bd = bd0 + (uint64_t)((ch * Cfg::CH_KV + in * 32u) >> 4);
-              ptx::mma_ss<Cfg::FP8>(d_t, ad, bd, Cfg::IDESC_QK, kk > 0 ? 1u : 0u);
-            }
-            ptx::tc_commit(bar(Cfg::B_SFULL + t * SB + j % SB));
-          };
-          auto issue_pv = [&]() -> bool {
-            const int jj = j - 1;
-            if (!(has_v && jj < n_kv[t])) return true;
-            const int si = t * SB + jj % SB;
-            if (!wait_bar<kRoleMma>(bar(Cfg::B_PFULL + si), (uint32_t)((jj / SB) & 1), wc, kSitePFull)) return false;
+        if constexpr (SB == 2) {
+          // S is double-buffered: the products for key tile j go first, so
+          // they run under the softmax of key tile j-1; then the P V of
+          // key tile j-1 as each tile's P is released
+          if (has_k) {
+            ok = wait_bar<kRoleMma>(bar(Cfg::B_KFULL + j % KST), (uint32_t)((j / KST) & 1), wc, kSiteKFull);
+            if (!ok) break;
             ptx::tc_fence_after();
-            const uint32_t d_t = tmem + (uint32_t)(Cfg::O_COL0 + t * D);
-            const uint32_t a_t = tmem + (uint32_t)(si * BN);
-            const uint64_t bd0 = ptx::sdesc_sw128(v_s + (jj % VST) * Cfg::KV_BYTES, Cfg::CH_KV, 1024u);
 #pragma unroll
-            for (int kk = 0; kk < Cfg::PV_STEPS; ++kk) {
-              const uint64_t bd = bd0 + (uint64_t)(((uint32_t)kk * Cfg::KSTEP * 128u) >> 4);
-              ptx::mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
-            }
-            ptx::tc_commit(bar(Cfg::B_ODONE + t));
-            return true;
-          };
-          if (SB == 2) {
-            issue_qk();
-            ok = issue_pv();
-          } else {
-            ok = issue_pv();
-            if (ok) issue_qk();
+            for (int t = 0; t < NQT; ++t)
+              if (j < n_kv[t]) issue_qk(t, j);
+            ptx::tc_commit(bar(Cfg::B_KEMPTY + j % KST));
+          }
+          if (has_v) {
+            ok = wait_bar<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc,
+                                    kSiteVFull);
+            if (!ok) break;
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int t = 0; t < NQT && ok; ++t)
+              if (j - 1 < n_kv[t]) ok = issue_pv(t, j - 1);
+            if (!ok) break;
+            ptx::tc_commit(bar(Cfg::B_VEMPTY + (j - 1) % VST));
+          }
+        } else {
+          // P overwrites S in place: PV(t, j-1) must be issued before
+          // QK(t, j) reuses the buffer
+          if (has_k) {
+            ok = wait_bar<kRoleMma>(bar(Cfg::B_KFULL + j % KST), (uint32_t)((j / KST) & 1), wc, kSiteKFull);
+            if (!ok) break;
+          }
+          if (has_v) {
+            ok = wait_bar<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc,
+                                    kSiteVFull);
+            if (!ok) break;
+          }
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int t = 0; t < NQT && ok; ++t) {
+            if (has_v && j - 1 < n_kv[t]) ok = issue_pv(t, j - 1);
+            if (ok && has_k && j < n_kv[t]) issue_qk(t, j);
           }
           if (!ok) break;
+          if (has_k) ptx::tc_commit(bar(Cfg::B_KEMPTY + j % KST));
+          if (has_v) ptx::tc_commit(bar(Cfg::B_VEMPTY + (j - 1) % VST));
         }
-        if (!ok) break;
-        if (has_k) ptx::tc_commit(bar(Cfg::B_KEMPTY + j % KST));
-        if (has_v) ptx::tc_commit(bar(Cfg::B_VEMPTY + (j - 1) % VST));
       }
       // All issued MMAs must finish before tensor memory is freed.
       ptx::tc_commit(bar(Cfg::B_DRAIN));

@@ -135,14 +135,19 @@ def test_key_permutation_invariance(d):
 
 @pytest.mark.parametrize("d", [64, 128, 256])
 def test_large_scores_and_dominant_key(d):
-    """Q x 30 pushes scores to ~1e3 (many rescales, one dominant key per row)."""
+    """Q x 30 pushes scores to ~1e3 (many rescales, one dominant key per row).
+    This is outside the N(0,1) condition the 1e-2 bar is stated for: a weight
+    near 1 rounded to bf16 (relative 2^-9) while the row sum keeps the fp32
+    weight moves O by up to 2^-9 |v| (|v| <= 4: 0.008), plus the output
+    rounding (0.008), so the max bound here is 2e-2."""
     qb, kb, vb = qkv(1, 2, 2, 257, 515, d)
     q30 = gen.f32_to_bf16_bits((f64(qb) * 30.0).astype(np.float32))
     for causal in (False, True):
         o, lse = run_attn(q30, kb, vb, causal)
         o_ref, lse_ref = oracle.attn_fwd(f64(q30), f64(kb), f64(vb), causal, 1 / math.sqrt(d))
         # LSE of scores ~1e3 in fp32: allow relative 1e-6 on top of the absolute bar
-        tol = dict(BF16_TOL, lse=max(BF16_TOL["lse"], 1e-6 * float(np.max(np.abs(lse_ref[np.isfinite(lse_ref)])))))
+        tol = dict(BF16_TOL, max_abs=2e-2,
+                   lse=max(BF16_TOL["lse"], 1e-6 * float(np.max(np.abs(lse_ref[np.isfinite(lse_ref)])))))
         compare(o, lse, o_ref, lse_ref, tol)
 
 
