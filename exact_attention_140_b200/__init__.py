@@ -18,7 +18,8 @@ import os
 __all__ = [
     "ATTN_BF16", "ATTN_FP8_E4M3", "AttnError", "attn_fwd", "attn_fwd_fp8", "attn_hadamard_quant_fp8",
     "attn_hadamard_quant_fp8_workspace_bytes", "attn_get_last_device_error", "attn_status_string",
-    "attn_kv_tile_count", "attn_tile_kind", "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attention", "lib_path", "EXPORTS",
+    "attn_kv_tile_count", "attn_tile_kind", "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attention",
+    "attn_hadamard_quant_fp8_noalloc", "lib_path", "EXPORTS",
 ]
 
 ATTN_BF16 = 0
@@ -33,7 +34,7 @@ lib_path = os.path.join(_HERE, "libattn.so")
 EXPORTS = (
     "attn_fwd", "attn_fwd_fp8", "attn_hadamard_quant_fp8", "attn_hadamard_quant_fp8_workspace_bytes",
     "attn_get_last_device_error", "attn_status_string", "attn_kv_tile_count", "attn_tile_kind",
-    "attn_debug_unsatisfied_wait", "attn_debug_exp2",
+    "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attn_hadamard_quant_fp8_noalloc",
 )
 
 if not os.path.exists(lib_path):
@@ -48,6 +49,8 @@ _lib.attn_fwd_fp8.argtypes = [_vp] * 5 + [_I] * 7 + [_F, _vp, _vp, _vp, _vp]
 _lib.attn_fwd_fp8.restype = _I
 _lib.attn_hadamard_quant_fp8.argtypes = [_vp, _vp, _vp, _vp, _LL, _I, _vp, _vp]
 _lib.attn_hadamard_quant_fp8.restype = _I
+_lib.attn_hadamard_quant_fp8_noalloc.argtypes = [_vp, _vp, _vp, _LL, _I, _vp, _vp]
+_lib.attn_hadamard_quant_fp8_noalloc.restype = _I
 _lib.attn_hadamard_quant_fp8_workspace_bytes.argtypes = []
 _lib.attn_hadamard_quant_fp8_workspace_bytes.restype = _LL
 _lib.attn_get_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint)]
@@ -119,6 +122,13 @@ def attn_hadamard_quant_fp8(x, x8, descale, workspace, rows, d, signs=None, stre
     rc = _lib.attn_hadamard_quant_fp8(_ptr(x), _ptr(x8), _ptr(descale), _ptr(workspace), int(rows), int(d),
                                       _ptr(signs), _stream(stream))
     return _check(rc, "attn_hadamard_quant_fp8", raise_on_error)
+
+
+def attn_hadamard_quant_fp8_noalloc(x, x8, descale, rows, d, signs=None, stream=None, raise_on_error=True):
+    """attn_hadamard_quant_fp8 with the library's own static scratch (no workspace)."""
+    rc = _lib.attn_hadamard_quant_fp8_noalloc(_ptr(x), _ptr(x8), _ptr(descale), int(rows), int(d), _ptr(signs),
+                                              _stream(stream))
+    return _check(rc, "attn_hadamard_quant_fp8_noalloc", raise_on_error)
 
 
 def attn_get_last_device_error(stream=None):

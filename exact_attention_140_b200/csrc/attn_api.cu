@@ -18,6 +18,13 @@ namespace attn {
 namespace {
 
 __device__ unsigned int g_err_word;     // device error word (bounded waits that ran out)
+
+// Scratch of attn_hadamard_quant_fp8_noalloc: a fixed 256-byte array that every
+// device loading this library holds until process exit.  Only word 0 (the
+// running absolute maximum) is used; the rest pads it to the 256 bytes the
+// workspace-taking entry point asks for.
+constexpr int kNoAllocScratchBytes = 256;
+static __device__ __align__(256) unsigned int g_noalloc_scratch[kNoAllocScratchBytes / 4];
 __device__ float g_unit_descale = 1.0f;  // descale used when attn_fwd is given e4m3 inputs
 
 constexpr int kMaxDevices = 64;
@@ -330,6 +337,44 @@ int attn_hadamard_quant_fp8(const void* x, void* x8, float* descale, void* works
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned int* amax = static_cast<unsigned int*>(workspace);
+  if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), s) != cudaSuccess) return ATTN_ERR_CUDA;
+  const long long blocks_needed = (rows + kPrepWarps - 1) / kPrepWarps;
+  const long long cap = (long long)st->num_sms * 16;
+  const unsigned grid = (unsigned)(blocks_needed < 1 ? 1 : (blocks_needed < cap ? blocks_needed : cap));
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  fp8_amax_kernel<<<grid, 32 * kPrepWarps, 0, s>>>(xb, rows, signs, amax);
+  fp8_quant_kernel<<<grid, 32 * kPrepWarps, 0, s>>>(xb, rows, signs, amax, static_cast<uint8_t*>(x8), descale);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_hadamard_quant_fp8_noalloc(const void* x, void* x8, float* descale, long long rows, int d,
+                                    const float* signs, void* stream) {
+  // Same checks as attn_hadamard_quant_fp8, minus the workspace.
+  if (rows < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != kPrepD) return ATTN_ERR_UNSUPPORTED;
+  if (x == nullptr || x8 == nullptr || descale == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x8) || !aligned16(signs) || (reinterpret_cast<uintptr_t>(descale) & 3u) != 0)
+    return ATTN_ERR_MISALIGNED;
+  // The scratch this call needs must fit the static array.
+  if (attn_hadamard_quant_fp8_workspace_bytes() > (long long)kNoAllocScratchBytes) return ATTN_ERR_UNSUPPORTED;
+  int dev = 0, rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
+  // Host code cannot use g_noalloc_scratch's name as a device address: look the
+  // address up once per device, with that device current (the first call on a
+  // device does this).
+  static unsigned int* scratch[kMaxDevices] = {};
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (scratch[dev] == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return ATTN_ERR_CUDA;
+      scratch[dev] = static_cast<unsigned int*>(ptr);
+    }
+  }
+  unsigned int* amax = scratch[dev];
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's maximum: clear it first.
   if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), s) != cudaSuccess) return ATTN_ERR_CUDA;
   const long long blocks_needed = (rows + kPrepWarps - 1) / kPrepWarps;
   const long long cap = (long long)st->num_sms * 16;

@@ -122,6 +122,30 @@ int attn_hadamard_quant_fp8(const void *x, void *x8, float *descale, void *works
 long long attn_hadamard_quant_fp8_workspace_bytes(void);
 
 /*
+ * attn_hadamard_quant_fp8_noalloc -- attn_hadamard_quant_fp8 without the
+ * workspace argument, for callers that cannot allocate device memory: code
+ * whose device memory is owned by another allocator it has no handle to, and
+ * real-time or plug-in code that must not call cudaMalloc on its hot path.
+ * The pages have no counterpart; this is a packaging of the same operation.
+ *   x, x8, descale, rows, d, signs, stream  as attn_hadamard_quant_fp8.
+ * Scratch: a 256-byte file-scope device array inside the library (every GPU
+ * that loads the library holds it until the process exits).  The call needs
+ * attn_hadamard_quant_fp8_workspace_bytes() of it (currently 256 bytes, for
+ * any rows); a build whose need exceeded 256 bytes would return
+ * ATTN_ERR_UNSUPPORTED.  Nothing is allocated: no cudaMalloc/cudaFree and no
+ * allocating library routine.
+ * Set-up: the first call on a device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ * Sharing: all calls on a device use the same array, which keeps the last
+ * call's contents; each call clears the part that must start at zero.  Calls
+ * that overlap on the GPU (for example on two streams) race on the array and
+ * must be ordered by the caller.
+ * Returns ATTN_OK or an error code, as attn_hadamard_quant_fp8.
+ */
+int attn_hadamard_quant_fp8_noalloc(const void *x, void *x8, float *descale, long long rows, int d,
+                                    const float *signs, void *stream);
+
+/*
  * attn_get_last_device_error -- synchronises `stream`, then reads and clears
  * the device error word of the current device.  Returns ATTN_OK,
  * ATTN_ERR_DEVICE_TIMEOUT (a bounded wait ran out inside a kernel) or
