@@ -11,6 +11,7 @@
 
 #include "attn.h"
 #include "attn_fwd_kernel.cuh"
+#include "attn_fwd_persistent_kernel.cuh"
 #include "fp8_prep.cuh"
 #include "tiles.h"
 
@@ -144,76 +145,114 @@ __global__ void exp2_probe_kernel(const float* x, float* y, long long n, int mod
   if (i + 1 < n) y[i + 1] = yb;
 }
 
+// Fills the parameters both kernels share; false when the work items do not
+// fit the kernels' int indexing.
+template <class Cfg>
+bool fill_params(FwdParams* p, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
+                 const float* dq, const float* dk, const float* dv, DeviceState* st) {
+  p->o = o;
+  p->lse = lse;
+  p->B = B;
+  p->Hq = Hq;
+  p->Hkv = Hkv;
+  p->Nq = Nq;
+  p->Nk = Nk;
+  p->group = Hq / Hkv;
+  p->n_qblocks = (Nq + Cfg::BM * Cfg::NQT - 1) / (Cfg::BM * Cfg::NQT);
+  const long long items = (long long)B * Hq * p->n_qblocks;
+  if (items > 0x7FFFFFFFll) return false;
+  p->n_items = (int)items;
+  // causal blocks differ in length: the persistent kernel orders them
+  // longest-first across heads when all of K and V fits comfortably in L2;
+  // otherwise it keeps a head's query blocks together so that they share its
+  // K/V tiles through L2
+  const long long kv_bytes = 2ll * B * Nk * Hkv * Cfg::D * Cfg::ELEM;
+  p->qb_major = (Cfg::CAUSAL && kv_bytes <= (48ll << 20)) ? 1 : 0;
+  p->sl2 = scale * 1.4426950408889634f;
+  p->dq = dq;
+  p->dk = dk;
+  p->dv = dv;
+  p->err = st->err;
+  p->timeout_ns = timeout_ns();
+  return true;
+}
+
+template <class Cfg>
+int encode_qkv(CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv, const void* q, const void* k, const void* v,
+               int B, int Hq, int Hkv, int Nq, int Nk) {
+  if (encode_bnhd(tq, q, Cfg::FP8, B, Nq, Hq, Cfg::D, Cfg::BM) != ATTN_OK ||
+      encode_bnhd(tk, k, Cfg::FP8, B, Nk, Hkv, Cfg::D, Cfg::BN) != ATTN_OK ||
+      encode_bnhd(tv, v, Cfg::FP8, B, Nk, Hkv, Cfg::D, Cfg::BN) != ATTN_OK)
+    return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+// Raises the kernel's dynamic shared memory limit once per device.
+template <class Kernel>
+int set_smem_once(Kernel kernel, int bytes, bool (&done)[kMaxDevices]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    done[dev] = true;
+  }
+  return ATTN_OK;
+}
+
+// One block per work item (batch, query head, query block).
 template <class Cfg>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
                int Nk, float scale, const float* dq, const float* dk, const float* dv, DeviceState* st,
                cudaStream_t stream) {
   static bool attr_set[kMaxDevices] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)Cfg::SMEM_BYTES) != cudaSuccess)
-      return ATTN_ERR_CUDA;
-    attr_set[dev] = true;
-  }
+  int rc = set_smem_once(attn_fwd_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set);
+  if (rc != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv;
-  if (encode_bnhd(&tq, q, Cfg::FP8, B, Nq, Hq, Cfg::D, Cfg::BM) != ATTN_OK ||
-      encode_bnhd(&tk, k, Cfg::FP8, B, Nk, Hkv, Cfg::D, Cfg::BN) != ATTN_OK ||
-      encode_bnhd(&tv, v, Cfg::FP8, B, Nk, Hkv, Cfg::D, Cfg::BN) != ATTN_OK)
-    return ATTN_ERR_CUDA;
+  if ((rc = encode_qkv<Cfg>(&tq, &tk, &tv, q, k, v, B, Hq, Hkv, Nq, Nk)) != ATTN_OK) return rc;
   FwdParams p;
-  p.o = o;
-  p.lse = lse;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.Nq = Nq;
-  p.Nk = Nk;
-  p.group = Hq / Hkv;
-  p.n_qblocks = (Nq + Cfg::BM * Cfg::NQT - 1) / (Cfg::BM * Cfg::NQT);
-  p.sl2 = scale * 1.4426950408889634f;
-  p.dq = dq;
-  p.dk = dk;
-  p.dv = dv;
-  p.err = st->err;
-  p.timeout_ns = timeout_ns();
+  if (!fill_params<Cfg>(&p, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st)) return ATTN_ERR_UNSUPPORTED;
   const dim3 grid((unsigned)p.n_qblocks, (unsigned)Hq, (unsigned)B);
   attn_fwd_kernel<Cfg><<<grid, Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// One block per SM, each looping over work items.
+template <class Cfg>
+int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                          int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
+                          DeviceState* st, cudaStream_t stream) {
+  static bool attr_set[kMaxDevices] = {};
+  int rc = set_smem_once(attn_fwd_persistent_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set);
+  if (rc != ATTN_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if ((rc = encode_qkv<Cfg>(&tq, &tk, &tv, q, k, v, B, Hq, Hkv, Nq, Nk)) != ATTN_OK) return rc;
+  FwdParams p;
+  if (!fill_params<Cfg>(&p, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st)) return ATTN_ERR_UNSUPPORTED;
+  const int nblk = p.n_items < st->num_sms ? p.n_items : st->num_sms;
+  attn_fwd_persistent_kernel<Cfg><<<dim3((unsigned)nblk), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Key ranges up to this length use the persistent kernel: their work items
+// are short, and a persistent block overlaps an item's fixed costs (first
+// loads, epilogue) with the neighbouring items instead of paying a block
+// start for each.  Longer items run one block per item.
+constexpr int kPersistentMaxNk = 1024;
+
 template <int D, int BN, int NQT, int KST, int VST, bool FP8, int EMU, int SB = (NQT == 1 ? 2 : 1)>
 int launch_causal(bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                   int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
                   DeviceState* st, cudaStream_t s) {
-  if (causal)
-    return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU, SB>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale,
-                                                                         dq, dk, dv, st, s);
-  return launch_fwd<FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU, SB>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale,
-                                                                        dq, dk, dv, st, s);
-}
-
-// Share of softmax exponentials computed in software (out of 8 element pairs);
-// ATTN_EMU overrides the built-in choice for tuning runs.
-int emu_setting(int dflt) {
-  static int v = [] {
-    const char* e = std::getenv("ATTN_EMU");
-    return e == nullptr ? -1 : std::atoi(e);
-  }();
-  return v < 0 ? dflt : v;
-}
-
-template <int D, int BN, int NQT, int KST, int VST, bool FP8>
-int launch_emu(int emu, bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B,
-               int Hq, int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
-               DeviceState* st, cudaStream_t s) {
-  switch (emu) {
-    case 0: return launch_causal<D, BN, NQT, KST, VST, FP8, 0>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
-    case 2: return launch_causal<D, BN, NQT, KST, VST, FP8, 2>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
-    case 4: return launch_causal<D, BN, NQT, KST, VST, FP8, 4>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
-    default: return launch_causal<D, BN, NQT, KST, VST, FP8, 3>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
+  const bool persist = Nk <= kPersistentMaxNk;
+  if (causal) {
+    using C = FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU, SB>;
+    return persist ? launch_fwd_persistent<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
+                   : launch_fwd<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
   }
+  using C = FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU, SB>;
+  return persist ? launch_fwd_persistent<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
+                 : launch_fwd<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
 }
 
 int check_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
@@ -294,12 +333,12 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
   const bool c = causal != 0;
   switch (d) {
-    case 64:
-      return launch_emu<64, 128, 2, 3, 3, false>(emu_setting(3), c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale,
-                                                 nullptr, nullptr, nullptr, st, s);
-    case 128:
-      return launch_emu<128, 128, 2, 2, 2, false>(emu_setting(2), c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale,
-                                                  nullptr, nullptr, nullptr, st, s);
+    case 64:  // 3 of 8 exponentials in software: at d = 64 the exponential costs twice the tensor time
+      return launch_causal<64, 128, 2, 3, 3, false, 3>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
+                                                       nullptr, nullptr, st, s);
+    case 128:  // 2 of 8 exponentials in software
+      return launch_causal<128, 128, 2, 2, 2, false, 2>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
+                                                        nullptr, nullptr, st, s);
     default: return launch_causal<256, 64, 1, 2, 2, false, 0>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
                                                              nullptr, nullptr, st, s);
   }
@@ -318,8 +357,8 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float*
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
-  return launch_emu<128, 128, 2, 3, 3, true>(emu_setting(3), causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk,
-                                             scale, descale_q, descale_k, descale_v, st, s);
+  return launch_causal<128, 128, 2, 3, 3, true, 3>(causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, scale,
+                                                    descale_q, descale_k, descale_v, st, s);
 }
 
 long long attn_hadamard_quant_fp8_workspace_bytes(void) { return 256; }

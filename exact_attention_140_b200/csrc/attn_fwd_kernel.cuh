@@ -44,136 +44,14 @@
 #include <cstdint>
 #include <type_traits>
 
+#include "attn_common.cuh"
 #include "exp2_soft.cuh"
 #include "ptx.cuh"
 #include "tiles.h"
 
 namespace attn {
 
-struct FwdParams {
-  void* o;          // [B, Nq, Hq, D] bf16
-  float* lse;       // [B, Hq, Nq] fp32 or nullptr
-  int B, Hq, Hkv, Nq, Nk;
-  int group;        // Hq / Hkv
-  int n_qblocks;    // ceil(Nq / (128 * NQT))
-  float sl2;        // scale * log2(e)
-  const float* dq;  // FP8 descales (device scalars), nullptr for bf16
-  const float* dk;
-  const float* dv;
-  unsigned int* err;            // device error word
-  unsigned long long timeout_ns;
-};
 
-constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
-
-template <int D_, int BN_, int NQT_, int KST_, int VST_, bool CAUSAL_, bool FP8_, int EMU_ = 0,
-          int SB_ = (NQT_ == 1 ? 2 : 1)>
-struct FwdCfg {
-  static constexpr int D = D_, BN = BN_, NQT = NQT_, KST = KST_, VST = VST_;
-  // software exp2 share on full tiles: element pairs with (pair % 8) < EMU
-  static constexpr int EMU = EMU_;
-  static constexpr bool CAUSAL = CAUSAL_, FP8 = FP8_;
-  static constexpr int BM = 128;
-  static constexpr int SB = SB_;  // score buffers per query tile
-  static_assert(SB == 1 || SB == 2, "one or two score buffers");
-  static constexpr int ELEM = FP8 ? 1 : 2;
-  static constexpr int NCH = D * ELEM / 128;  // 128-byte column chunks per row
-  static constexpr int BOXE = 128 / ELEM;     // elements per chunk row
-  static constexpr uint32_t CH_Q = BM * 128;  // bytes of one chunk of a Q tile
-  static constexpr uint32_t CH_KV = BN * 128;
-  static constexpr uint32_t QT_BYTES = CH_Q * NCH;
-  static constexpr uint32_t KV_BYTES = CH_KV * NCH;
-  static constexpr int KSTEP = FP8 ? 32 : 16;  // reduction depth of one MMA
-  static constexpr int QK_STEPS = D / KSTEP;
-  static constexpr int PV_STEPS = BN / KSTEP;
-  static constexpr int P_COLS = BN * ELEM / 4;
-  static constexpr int O_COL0 = NQT * SB * BN;
-  static constexpr int TMEM_USED = O_COL0 + NQT * D;
-  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
-  static_assert(TMEM_USED <= 512, "tensor memory has 512 columns");
-  static_assert(D % 64 == 0 && NCH >= 1, "head size");
-  static_assert(BN % 32 == 0 && BN <= 256, "key tile");
-  // barriers
-  static constexpr int B_QFULL = 0;
-  static constexpr int B_KFULL = B_QFULL + NQT;
-  static constexpr int B_KEMPTY = B_KFULL + KST;
-  static constexpr int B_VFULL = B_KEMPTY + KST;
-  static constexpr int B_VEMPTY = B_VFULL + VST;
-  static constexpr int B_SFULL = B_VEMPTY + VST;
-  static constexpr int B_PFULL = B_SFULL + NQT * SB;
-  static constexpr int B_ODONE = B_PFULL + NQT * SB;
-  static constexpr int B_OFINAL = B_ODONE + NQT;
-  static constexpr int B_DRAIN = B_OFINAL + NQT;
-  static constexpr int NBAR = B_DRAIN + 1;
-  // shared memory (offsets from a 1024-byte aligned base)
-  static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + NQT * QT_BYTES;
-  static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + VST * KV_BYTES;
-  static constexpr uint32_t OFF_SLOT = OFF_BAR + NBAR * 8;
-  static constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
-  static constexpr uint32_t SMEM_BYTES = OFF_ABORT + 4 + 1024;
-  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per block");
-  // warps: softmax warpgroups, then one warpgroup holding the TMA warp, the
-  // MMA warp and two idle warps (a whole warpgroup, so that registers can be
-  // moved to the softmax warpgroups with setmaxnreg)
-  static constexpr int SM_WARPS = 4 * NQT;
-  static constexpr int TMA_WARP = SM_WARPS;
-  static constexpr int MMA_WARP = SM_WARPS + 1;
-  static constexpr int NTHREADS = 32 * (SM_WARPS + 4);
-  // register split (NQT = 2: 384 threads launch with 168 registers each =
-  // 64512; softmax warpgroups get 224, the control warpgroup keeps 56:
-  // 2*128*224 + 128*56 = 64512)
-  static constexpr int REG_LAUNCH = 65536 / NTHREADS >= 255 ? 255 : (65536 / NTHREADS) / 8 * 8;
-  static constexpr bool SPLIT_REGS = NQT == 2;
-  static constexpr int REG_SOFTMAX = 200, REG_CONTROL = 104;
-  static_assert(!SPLIT_REGS || 2 * 128 * REG_SOFTMAX + 128 * REG_CONTROL <= NTHREADS * REG_LAUNCH,
-                "register split exceeds the launch allocation");
-  static constexpr uint32_t IDESC_QK = ptx::idesc<FP8>(128, BN, false);
-  static constexpr uint32_t IDESC_PV = ptx::idesc<FP8>(128, D, true);
-};
-
-// Wait sites recorded in the device error word.
-enum : uint32_t {
-  kSiteQ = 1, kSiteKFull, kSiteVFull, kSiteKEmpty, kSiteVEmpty, kSiteSFull, kSitePFull,
-  kSiteODone, kSiteDrain, kSiteProbe
-};
-
-struct WaitCtx {
-  volatile uint32_t* abort;
-  unsigned int* err;
-  unsigned long long timeout_ns;
-};
-
-// Bounded mbarrier wait: true when the phase with `parity` has completed;
-// false after the time limit (recording the site in the error word and
-// raising the block's abort flag) or when another role already aborted.
-// The first probe is inline; only a wait that does not succeed at once pays
-// for the call into the polling loop.  The polling loop is instantiated once
-// per warp role (ROLE), because roles run under different register budgets
-// (setmaxnreg) and a called function is compiled for one budget.
-template <int ROLE>
-__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, const WaitCtx& c, uint32_t site) {
-  const uint64_t t0 = ptx::globaltimer();
-  for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 16; ++i)
-      if (ptx::mbar_try_wait(bar, parity)) return true;
-    if (*c.abort) return false;
-    if (ptx::globaltimer() - t0 > c.timeout_ns) {
-      *c.abort = 1u;
-      const uint32_t blk = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
-      atomicOr(c.err, 1u | (site << 8) | ((blk & 0xFFFFu) << 16));
-      return false;
-    }
-  }
-}
-template <int ROLE = 0>
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const WaitCtx& c, uint32_t site) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  return wait_bar_slow<ROLE>(bar, parity, c, site);
-}
-enum : int { kRoleSoftmax = 0, kRoleProducer = 1, kRoleMma = 2 };
 
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::NTHREADS, 1)

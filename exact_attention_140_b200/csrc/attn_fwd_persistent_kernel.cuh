@@ -1,0 +1,580 @@
+// attn_fwd_persistent_kernel.cuh -- persistent variant of the fused
+// attention forward, for short key ranges.
+//
+// It computes the same thing as attn_fwd_kernel (same tiles, warp roles,
+// tensor-memory layout, online softmax with lazy rescaling and epilogue; see
+// that file), but a grid of one block per SM loops over the work items
+// (batch, query head, query block) instead of launching one block per item.
+// With short key ranges an item is only a few key tiles long and the fixed
+// costs around it -- block start, tensor-memory allocation, the first Q and
+// K/V loads, the epilogue's read-out of O -- are a large share of its time;
+// here they overlap with the neighbouring items:
+//   * the producer issues the next item's first K/V tile while the current
+//     item is still computing, and its Q tile as soon as the last Q K^T of
+//     the current item has completed (barrier q_empty);
+//   * the MMA warp starts the next item's products while the softmax
+//     warpgroups write out the previous output; only its first P V waits
+//     for that output's read-out (barrier o_free);
+//   * each P is released in two halves (barrier p_half): the P V over the
+//     first half of the keys starts while the second half is exponentiated.
+// Ring slots and barrier phases are counted across items, so the pipeline
+// never drains between them.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include <type_traits>
+
+#include "attn_common.cuh"
+#include "exp2_soft.cuh"
+#include "ptx.cuh"
+#include "tiles.h"
+
+namespace attn {
+
+// Work items are (batch, query head, query block).  The grid is persistent
+// (one block per SM); block c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... of an
+// order sorted longest-first (for causal masks), so long and short items pair
+// up.  Head-major order keeps the query blocks of one head on the GPU at the
+// same time (their K/V tiles are shared through L2).
+__device__ __forceinline__ int item_at(int k, int G, int T) {
+  const int c = (int)blockIdx.x;
+  const long long pos = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
+  return pos < T ? (int)pos : -1;
+}
+struct Item {
+  int qb, h, b;
+};
+__device__ __forceinline__ Item decode_item(int i, const FwdParams& p) {
+  const int bh = p.B * p.Hq;
+  int qr, r;
+  if (p.qb_major) {
+    qr = i / bh;
+    r = i - qr * bh;
+  } else {
+    r = i / p.n_qblocks;
+    qr = i - r * p.n_qblocks;
+  }
+  return Item{p.n_qblocks - 1 - qr, r % p.Hq, r / p.Hq};
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::NTHREADS, 1)
+    attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  constexpr int BM = Cfg::BM, BN = Cfg::BN, D = Cfg::D, NQT = Cfg::NQT, SB = Cfg::SB;
+  constexpr int KST = Cfg::KST, VST = Cfg::VST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
+  const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw_u32);
+  auto bar = [&](int i) -> uint32_t { return sbase + Cfg::OFF_BAR + 8u * (uint32_t)i; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sgen + Cfg::OFF_ABORT);
+  const WaitCtx wc{abort_flag, p.err, p.timeout_ns};
+  const int G = (int)gridDim.x, T = p.n_items;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // key tiles the query tiles of an item visit (0 = none)
+  auto plan = [&](const Item& it, int (&n_kv)[NQT]) -> int {
+    const int q0 = it.qb * BM * NQT;
+    int nmax = 0;
+#pragma unroll
+    for (int t = 0; t < NQT; ++t) {
+      n_kv[t] = kv_tile_count(q0 + t * BM, q0 + (t + 1) * BM, p.Nq, p.Nk, BN, Cfg::CAUSAL);
+      nmax = n_kv[t] > nmax ? n_kv[t] : nmax;
+    }
+    return nmax;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < NQT; ++t) ptx::mbar_init(bar(Cfg::B_QFULL + t), 1);
+    for (int s = 0; s < KST; ++s) {
+      ptx::mbar_init(bar(Cfg::B_KFULL + s), 1);
+      ptx::mbar_init(bar(Cfg::B_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < VST; ++s) {
+      ptx::mbar_init(bar(Cfg::B_VFULL + s), 1);
+      ptx::mbar_init(bar(Cfg::B_VEMPTY + s), 1);
+    }
+    for (int i = 0; i < NQT * SB; ++i) {
+      ptx::mbar_init(bar(Cfg::B_SFULL + i), 1);
+      ptx::mbar_init(bar(Cfg::B_PFULL + i), 128);
+      ptx::mbar_init(bar(Cfg::B_PHALF + i), 128);
+    }
+    for (int t = 0; t < NQT; ++t) {
+      ptx::mbar_init(bar(Cfg::B_ODONE + t), 1);
+      ptx::mbar_init(bar(Cfg::B_OFINAL + t), 1);
+      ptx::mbar_init(bar(Cfg::B_OFREE + t), 128);
+    }
+    ptx::mbar_init(bar(Cfg::B_QEMPTY), 1);
+    ptx::mbar_init(bar(Cfg::B_DRAIN), 1);
+    *abort_flag = 0u;
+    ptx::fence_mbar_init();
+  }
+  if (warp == Cfg::TMA_WARP && lane == 0) {
+    ptx::prefetch_tmap(&tmQ);
+    ptx::prefetch_tmap(&tmK);
+    ptx::prefetch_tmap(&tmV);
+  }
+  if (warp == Cfg::MMA_WARP) {
+    ptx::tmem_alloc(sbase + Cfg::OFF_SLOT, Cfg::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sgen + Cfg::OFF_SLOT);
+
+  if (warp < Cfg::SM_WARPS) {
+    // ------------------------------------------------------------ softmax
+    if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_inc<Cfg::REG_SOFTMAX>();
+    const int t = warp >> 2, wq = warp & 3;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t o_taddr = tmem + lane_off + (uint32_t)(Cfg::O_COL0 + t * D);
+    float sl2 = p.sl2;
+    if constexpr (Cfg::FP8) sl2 *= __ldg(p.dq) * __ldg(p.dk);
+    int scount = 0;       // score buffers of this query tile consumed so far (= P V products issued before)
+    int finals = 0;       // items whose output this tile has written
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int item = item_at(k, G, T);
+      if (item < 0) break;
+      const Item it = decode_item(item, p);
+      int n_kv[NQT];
+      plan(it, n_kv);
+      const int row0 = it.qb * BM * NQT + t * BM;
+      const int row = row0 + wq * 32 + lane;
+      const int nt = n_kv[t];
+      const int vend = (int)vis_end(row, p.Nq, p.Nk, Cfg::CAUSAL);
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < nt; ++j, ++scount) {
+        const int si = t * SB + (scount % SB);
+        ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_SFULL + si), (uint32_t)((scount / SB) & 1), wc, kSiteSFull);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint32_t s_taddr = tmem + lane_off + (uint32_t)(si * BN);
+        const bool partial = tile_kind(row0, row0 + BM, j, p.Nq, p.Nk, BN, Cfg::CAUSAL) == kTilePartial;
+        const int nvis = vend - j * BN;  // visible keys of this tile (masks partial tiles)
+        // ---- one read of the whole score row (one TMEM load latency per tile)
+        uint32_t sr[BN];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c)
+          ptx::tmem_ld32(s_taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) ptx::tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+        float m_blk;
+        if (partial) {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < BN; ++c) mx = fmaxf(mx, (c < nvis) ? __uint_as_float(sr[c]) * sl2 : -INFINITY);
+          m_blk = mx;
+        } else if (sl2 >= 0.f) {
+          float a0 = __uint_as_float(sr[0]), a1 = __uint_as_float(sr[1]);
+          float a2 = __uint_as_float(sr[2]), a3 = __uint_as_float(sr[3]);
+#pragma unroll
+          for (int c = 4; c < BN; c += 8) {
+            a0 = ptx::fmax3(a0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+            a1 = ptx::fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+            if (c + 4 < BN) {
+              a2 = ptx::fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+              a3 = ptx::fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+            }
+          }
+          m_blk = ptx::fmax3(a0, a1, fmaxf(a2, a3)) * sl2;
+        } else {  // a negative scale turns the row max into the row min
+          float mn = __uint_as_float(sr[0]);
+#pragma unroll
+          for (int c = 1; c < BN; ++c) mn = fminf(mn, __uint_as_float(sr[c]));
+          m_blk = mn * sl2;
+        }
+        float alpha = 1.f;
+        bool resc = false;
+        if (m_blk > m_ref + kTau) {
+          alpha = ptx::ex2(m_ref - m_blk);  // 0 when m_ref = -inf
+          resc = (m_ref != -INFINITY);
+          m_ref = m_blk;
+          l *= alpha;
+        }
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const bool resc_any = __any_sync(0xffffffffu, resc);
+        // ---- exponentiate 32 columns at a time; each chunk's packed P is
+        // stored at once (over score columns already read), so the registers
+        // of a chunk die before the next chunk is processed
+        uint64_t lsum[4] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
+        const uint64_t sl2x2 = ptx::f2(sl2, sl2), negm2 = ptx::f2(-m_use, -m_use);
+        constexpr int PW = Cfg::FP8 ? 8 : 16;  // packed P words per 32 scores
+        // The tile kind is resolved once, outside the unrolled loop: one loop
+        // body per kind, no per-element branches.
+        auto exp_row = [&](auto partial_tag) {
+          constexpr bool PARTIAL = decltype(partial_tag)::value;
+#pragma unroll
+          for (int ch = 0; ch < BN / 32; ++ch) {
+            uint32_t pk[PW];
+            [[maybe_unused]] float hold0 = 0.f, hold1 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int col = 32 * ch + 2 * c;
+              const float s0 = __uint_as_float(sr[col]), s1 = __uint_as_float(sr[col + 1]);
+              float e0, e1;
+              if constexpr (PARTIAL) {
+                e0 = ptx::ex2((col < nvis ? s0 * sl2 : -INFINITY) - m_use);
+                e1 = ptx::ex2((col + 1 < nvis ? s1 * sl2 : -INFINITY) - m_use);
+              } else {
+                const uint64_t x = ptx::ffma2(ptx::f2(s0, s1), sl2x2, negm2);
+                float x0, x1;
+                ptx::unf2(x, x0, x1);
+                if (((16 * ch + c) % 8) < Cfg::EMU) {
+                  exp2_soft2(x0, x1, e0, e1);
+                } else {
+                  e0 = ptx::ex2(x0);
+                  e1 = ptx::ex2(x1);
+                }
+              }
+              lsum[c % 4] = ptx::fadd2(lsum[c % 4], ptx::f2(e0, e1));
+              if constexpr (Cfg::FP8) {
+                if (c % 2 == 0) {
+                  hold0 = e0;
+                  hold1 = e1;
+                } else {
+                  pk[c / 2] = ptx::pack_e4m3x4(hold0, hold1, e0, e1);
+                }
+              } else {
+                pk[c] = ptx::pack_bf16x2(e0, e1);
+              }
+            }
+            if constexpr (Cfg::FP8)
+              ptx::tmem_st8(s_taddr + (uint32_t)(PW * ch), pk);
+            else
+              ptx::tmem_st16(s_taddr + (uint32_t)(PW * ch), pk);
+            if (ch == BN / 64 - 1 && !resc_any) {
+              // the first half of P is in TMEM: its P V can start while the
+              // second half is exponentiated (a warp that must rescale O
+              // first releases it after the rescale instead)
+              ptx::tmem_wait_st();
+              ptx::tc_fence_before();
+              ptx::mbar_arrive(bar(Cfg::B_PHALF + si));
+            }
+          }
+        };
+        if (partial)
+          exp_row(std::true_type{});
+        else
+          exp_row(std::false_type{});
+        {
+          float la, lb;
+          ptx::unf2(ptx::fadd2(ptx::fadd2(lsum[0], lsum[1]), ptx::fadd2(lsum[2], lsum[3])), la, lb);
+          l += la + lb;
+        }
+        ptx::tmem_wait_st();
+        if (resc_any) {
+          // O_t must hold exactly the products of key tiles < j: wait for
+          // PV(t, j-1), the (scount - 1)-th product of this tile (one product
+          // per score tile).  Whenever S(t, j) is ready the product before
+          // that one has completed (it was issued before QK(t, j)) and PV(t, j)
+          // is not issued yet, so the o_done barrier is within one phase of
+          // the target and the parity test is unambiguous.
+          ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_ODONE + t), (uint32_t)((scount - 1) & 1), wc, kSiteODone);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          const float a = resc ? alpha : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(o_taddr + 32 * c, r);
+            ptx::tmem_wait_ld_dep(r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * a);
+            ptx::tmem_st32(o_taddr + 32 * c, r);
+          }
+          ptx::tmem_wait_st();
+        }
+        ptx::tc_fence_before();
+        if (resc_any) ptx::mbar_arrive(bar(Cfg::B_PHALF + si));
+        ptx::mbar_arrive(bar(Cfg::B_PFULL + si));
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      if (nt > 0) {  // o_final completes once per item, after the tile's last PV
+        ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_OFINAL + t), (uint32_t)(finals & 1), wc, kSiteODone);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++finals;
+      }
+      ptx::tc_fence_after();
+      const bool store = row < p.Nq;
+      float inv = l > 0.f ? 1.f / l : 0.f;
+      if constexpr (Cfg::FP8) inv *= __ldg(p.dv);
+      const Item ie = decode_item(item, p);  // recomputed: keeps fewer values live through the key loop
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
+                            (((long long)ie.b * p.Nq + row) * p.Hq + ie.h) * (long long)D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        if (nt > 0) {
+          ptx::tmem_ld32(o_taddr + 32 * c, r);
+          ptx::tmem_wait_ld_dep(r);
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = nt > 0 ? ptx::pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv)
+                        : 0u;
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+      if (nt > 0) {  // O of this tile is read out: the next item may overwrite it
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(Cfg::B_OFREE + t));
+      }
+      if (store && p.lse != nullptr) {
+        const float lse = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        p.lse[((long long)ie.b * p.Hq + ie.h) * p.Nq + row] = lse;
+      }
+    }
+  } else if (warp == Cfg::TMA_WARP) {
+    // ------------------------------------------------------------ producer
+    if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_dec<Cfg::REG_CONTROL>();
+    if (lane == 0) {
+      int k_issued[KST], v_issued[VST], q_issued[NQT];
+#pragma unroll
+      for (int s = 0; s < KST; ++s) k_issued[s] = 0;
+#pragma unroll
+      for (int s = 0; s < VST; ++s) v_issued[s] = 0;
+#pragma unroll
+      for (int t = 0; t < NQT; ++t) q_issued[t] = 0;
+      int kc = 0, vc = 0;  // loads issued into the K and V rings
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int item = item_at(k, G, T);
+        if (item < 0) break;
+        const Item it = decode_item(item, p);
+        int n_kv[NQT];
+        const int nmax = plan(it, n_kv);
+        const int kh = it.h / p.group;
+        const int q0 = it.qb * BM * NQT;
+        auto load_kv = [&](int j) -> bool {
+          const int ks = kc % KST;
+          if (kc >= KST &&
+              !wait_bar<kRoleProducer>(bar(Cfg::B_KEMPTY + ks), (uint32_t)(((kc / KST) - 1) & 1), wc, kSiteKEmpty))
+            return false;
+          {
+            const uint32_t fb = bar(Cfg::B_KFULL + ks);
+            ptx::mbar_arrive_expect_tx(fb, Cfg::KV_BYTES);
+#pragma unroll
+            for (int c = 0; c < Cfg::NCH; ++c)
+              ptx::tma_load_4d(sbase + Cfg::OFF_K + ks * Cfg::KV_BYTES + c * Cfg::CH_KV, &tmK, fb, c * Cfg::BOXE, kh,
+                               j * BN, it.b);
+            ++k_issued[ks];
+            ++kc;
+          }
+          const int vs = vc % VST;
+          if (vc >= VST &&
+              !wait_bar<kRoleProducer>(bar(Cfg::B_VEMPTY + vs), (uint32_t)(((vc / VST) - 1) & 1), wc, kSiteVEmpty))
+            return false;
+          {
+            const uint32_t fb = bar(Cfg::B_VFULL + vs);
+            ptx::mbar_arrive_expect_tx(fb, Cfg::KV_BYTES);
+#pragma unroll
+            for (int c = 0; c < Cfg::NCH; ++c)
+              ptx::tma_load_4d(sbase + Cfg::OFF_V + vs * Cfg::KV_BYTES + c * Cfg::CH_KV, &tmV, fb, c * Cfg::BOXE, kh,
+                               j * BN, it.b);
+            ++v_issued[vs];
+            ++vc;
+          }
+          return true;
+        };
+        // the first key/value tile goes out before waiting for Q smem, so it
+        // is in flight while the previous item finishes
+        if (nmax > 0 && !load_kv(0)) break;
+        // Q smem is free once the previous item's last Q K^T has completed
+        if (k > 0 && !wait_bar<kRoleProducer>(bar(Cfg::B_QEMPTY), (uint32_t)((k - 1) & 1), wc, kSiteQ)) break;
+#pragma unroll
+        for (int t = 0; t < NQT; ++t) {
+          if (n_kv[t] == 0) continue;
+          const uint32_t fb = bar(Cfg::B_QFULL + t);
+          ptx::mbar_arrive_expect_tx(fb, Cfg::QT_BYTES);
+#pragma unroll
+          for (int c = 0; c < Cfg::NCH; ++c)
+            ptx::tma_load_4d(sbase + Cfg::OFF_Q + t * Cfg::QT_BYTES + c * Cfg::CH_Q, &tmQ, fb, c * Cfg::BOXE, it.h,
+                             q0 + t * BM, it.b);
+          ++q_issued[t];
+        }
+        for (int j = 1; j < nmax; ++j)
+          if (!load_kv(j)) {
+            ok = false;
+            break;
+          }
+      }
+      // Every issued copy must land before the block may exit (no-op in the
+      // normal path, where the consumers have already seen them all).
+#pragma unroll
+      for (int t = 0; t < NQT; ++t)
+        if (q_issued[t] > 0)
+          wait_bar<kRoleProducer>(bar(Cfg::B_QFULL + t), (uint32_t)((q_issued[t] - 1) & 1), wc, kSiteQ);
+#pragma unroll
+      for (int s = 0; s < KST; ++s)
+        if (k_issued[s] > 0)
+          wait_bar<kRoleProducer>(bar(Cfg::B_KFULL + s), (uint32_t)((k_issued[s] - 1) & 1), wc, kSiteKFull);
+#pragma unroll
+      for (int s = 0; s < VST; ++s)
+        if (v_issued[s] > 0)
+          wait_bar<kRoleProducer>(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
+    }
+  } else {
+    if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_dec<Cfg::REG_CONTROL>();
+  }
+  if (warp == Cfg::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      const uint32_t q_s = sbase + Cfg::OFF_Q, k_s = sbase + Cfg::OFF_K, v_s = sbase + Cfg::OFF_V;
+      int kc = 0, vc = 0;                  // K / V ring slots consumed
+      int scount[NQT], pcount[NQT], qcount[NQT], ouse[NQT];
+#pragma unroll
+      for (int t = 0; t < NQT; ++t) scount[t] = pcount[t] = qcount[t] = ouse[t] = 0;
+      auto issue_qk = [&](int t, int kslot) {
+        const int buf = scount[t] % SB;
+        const uint32_t d_t = tmem + (uint32_t)((t * SB + buf) * BN);
+        // descriptors advance by 32 bytes (>> 4 = 2) per K step inside a
+        // 128-byte chunk and by one chunk (CH_Q / CH_KV bytes) after four
+        const uint64_t ad0 = ptx::sdesc_sw128(q_s + t * Cfg::QT_BYTES, 16u, 1024u);
+        const uint64_t bd0 = ptx::sdesc_sw128(k_s + kslot * Cfg::KV_BYTES, 16u, 1024u);
+#pragma unroll
+        for (int kk = 0; kk < Cfg::QK_STEPS; ++kk) {
+          const uint32_t ch = (uint32_t)kk / 4u, in = (uint32_t)kk % 4u;
+          const uint64_t ad = ad0 + (uint64_t)((ch * Cfg::CH_Q + in * 32u) >> 4);
+          const uint64_t bd = bd0 + (uint64_t)((ch * Cfg::CH_KV + in * 32u) >> 4);
+          ptx::mma_ss<Cfg::FP8>(d_t, ad, bd, Cfg::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        ptx::tc_commit(bar(Cfg::B_SFULL + t * SB + buf));
+        ++scount[t];
+      };
+      // P V of key tile jj of the current item; jj == 0 starts a new output
+      auto issue_pv = [&](int t, int jj, int vslot, bool last) -> bool {
+        if (jj == 0) {
+          // the previous item's output of this tile must have been read out
+          if (ouse[t] > 0 &&
+              !wait_bar<kRoleMma>(bar(Cfg::B_OFREE + t), (uint32_t)((ouse[t] - 1) & 1), wc, kSiteODone))
+            return false;
+          ++ouse[t];
+        }
+        const int buf = pcount[t] % SB;
+        const int si = t * SB + buf;
+        const uint32_t ph = (uint32_t)((pcount[t] / SB) & 1);
+        const uint32_t d_t = tmem + (uint32_t)(Cfg::O_COL0 + t * D);
+        const uint32_t a_t = tmem + (uint32_t)(si * BN);
+        const uint64_t bd0 = ptx::sdesc_sw128(v_s + vslot * Cfg::KV_BYTES, Cfg::CH_KV, 1024u);
+        // the first half of the keys as soon as their P is written, the rest
+        // when the whole P is
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (!wait_bar<kRoleMma>(bar((half == 0 ? Cfg::B_PHALF : Cfg::B_PFULL) + si), ph, wc, kSitePFull))
+            return false;
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int kk = half * Cfg::PV_STEPS / 2; kk < (half + 1) * Cfg::PV_STEPS / 2; ++kk) {
+            const uint64_t bd = bd0 + (uint64_t)(((uint32_t)kk * Cfg::KSTEP * 128u) >> 4);
+            ptx::mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        ptx::tc_commit(bar(Cfg::B_ODONE + t));
+        if (last) ptx::tc_commit(bar(Cfg::B_OFINAL + t));
+        ++pcount[t];
+        return true;
+      };
+      for (int k = 0; ok; ++k) {
+        const int item = item_at(k, G, T);
+        if (item < 0) break;
+        const Item it = decode_item(item, p);
+        int n_kv[NQT];
+        const int nmax = plan(it, n_kv);
+#pragma unroll
+        for (int t = 0; t < NQT && ok; ++t)
+          if (n_kv[t] > 0) {
+            ok = wait_bar<kRoleMma>(bar(Cfg::B_QFULL + t), (uint32_t)(qcount[t] & 1), wc, kSiteQ);
+            ++qcount[t];
+          }
+        if (!ok) break;
+        ptx::tc_fence_after();
+        for (int j = 0; ok && j <= nmax; ++j) {
+          const bool has_k = j < nmax, has_v = j >= 1;
+          const int ks = kc % KST, vs = vc % VST;
+          if constexpr (SB == 2) {
+            // S is double-buffered: the products for key tile j go first, so
+            // they run under the softmax of key tile j-1; then the P V of
+            // key tile j-1 as each tile's P is released
+            if (has_k) {
+              ok = wait_bar<kRoleMma>(bar(Cfg::B_KFULL + ks), (uint32_t)((kc / KST) & 1), wc, kSiteKFull);
+              if (!ok) break;
+              ptx::tc_fence_after();
+#pragma unroll
+              for (int t = 0; t < NQT; ++t)
+                if (j < n_kv[t]) issue_qk(t, ks);
+              ptx::tc_commit(bar(Cfg::B_KEMPTY + ks));
+              ++kc;
+            }
+            if (has_v) {
+              ok = wait_bar<kRoleMma>(bar(Cfg::B_VFULL + vs), (uint32_t)((vc / VST) & 1), wc, kSiteVFull);
+              if (!ok) break;
+              ptx::tc_fence_after();
+#pragma unroll
+              for (int t = 0; t < NQT && ok; ++t)
+                if (j - 1 < n_kv[t]) ok = issue_pv(t, j - 1, vs, j == n_kv[t]);
+              if (!ok) break;
+              ptx::tc_commit(bar(Cfg::B_VEMPTY + vs));
+              ++vc;
+            }
+          } else {
+            // P overwrites S in place: PV(t, j-1) must be issued before
+            // QK(t, j) reuses the buffer
+            if (has_k) {
+              ok = wait_bar<kRoleMma>(bar(Cfg::B_KFULL + ks), (uint32_t)((kc / KST) & 1), wc, kSiteKFull);
+              if (!ok) break;
+            }
+            if (has_v) {
+              ok = wait_bar<kRoleMma>(bar(Cfg::B_VFULL + vs), (uint32_t)((vc / VST) & 1), wc, kSiteVFull);
+              if (!ok) break;
+            }
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int t = 0; t < NQT && ok; ++t) {
+              if (has_v && j - 1 < n_kv[t]) ok = issue_pv(t, j - 1, vs, j == n_kv[t]);
+              if (ok && has_k && j < n_kv[t]) issue_qk(t, ks);
+            }
+            if (!ok) break;
+            if (has_k) {
+              ptx::tc_commit(bar(Cfg::B_KEMPTY + ks));
+              ++kc;
+            }
+            if (has_v) {
+              ptx::tc_commit(bar(Cfg::B_VEMPTY + vs));
+              ++vc;
+            }
+          }
+          // after the item's last Q K^T: Q smem is free once it completes,
+          // so the next item's Q can load under this item's last P V
+          if (j == nmax - 1) ptx::tc_commit(bar(Cfg::B_QEMPTY));
+        }
+        if (nmax == 0) ptx::tc_commit(bar(Cfg::B_QEMPTY));
+      }
+      // All issued MMAs must finish before tensor memory is freed.
+      ptx::tc_commit(bar(Cfg::B_DRAIN));
+      wait_bar<kRoleMma>(bar(Cfg::B_DRAIN), 0u, wc, kSiteDrain);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == Cfg::MMA_WARP) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

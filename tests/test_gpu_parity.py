@@ -61,10 +61,20 @@ def test_gqa_mqa_against_oracle(Hq, Hkv):
     full_check(2, Hq, Hkv, 257, 257, 128, True)
 
 
+# Key ranges up to 1024 run on the persistent kernel, longer ones on the
+# one-block-per-item kernel; these cases sit on both sides of that boundary.
 @pytest.mark.parametrize("d", [64, 128, 256])
-def test_gqa_equals_repeated_heads_bitwise(d):
+@pytest.mark.parametrize("Nq,Nk", [(1024, 1024), (300, 1025), (1100, 1100), (129, 1500)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_both_schedules(d, Nq, Nk, causal):
+    full_check(1, 2, 1, Nq, Nk, d, causal)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("N", [200, 1100])
+def test_gqa_equals_repeated_heads_bitwise(d, N):
     """Grouped heads read the shared K/V head: identical to MHA on repeated K/V."""
-    qb, kb, vb = qkv(1, 8, 2, 200, 200, d)
+    qb, kb, vb = qkv(1, 8, 2, N, N, d)
     o1, l1 = run_attn(qb, kb, vb, True)
     o2, l2 = run_attn(qb, np.repeat(kb, 4, axis=2), np.repeat(vb, 4, axis=2), True)
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
@@ -170,8 +180,9 @@ def test_empty_key_set():
     assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
 
 
-def test_repeatable():
-    qb, kb, vb = qkv(2, 4, 4, 512, 512, 128)
+@pytest.mark.parametrize("N", [512, 1300])
+def test_repeatable(N):
+    qb, kb, vb = qkv(2, 4, 4, N, N, 128)
     a = run_attn(qb, kb, vb, True)
     b = run_attn(qb, kb, vb, True)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
