@@ -342,7 +342,7 @@ def run_ours(args, cfg, name):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peaks['src']} {'bf16 x2 (fp8 nominal ratio)' if fp8 else 'bf16'}",
-                     "kernel": "attn_fwd_kernel"},
+                     "kernel": "attn_fwd_persistent_kernel" if ea.attn_fwd_schedule(N) == 1 else "attn_fwd_kernel"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in host)),
                 "d2h_bytes_per_step": int(o.numel() * o.element_size() + lse.numel() * lse.element_size())},

@@ -19,6 +19,7 @@ __all__ = [
     "ATTN_BF16", "ATTN_FP8_E4M3", "AttnError", "attn_fwd", "attn_fwd_fp8", "attn_hadamard_quant_fp8",
     "attn_hadamard_quant_fp8_workspace_bytes", "attn_get_last_device_error", "attn_status_string",
     "attn_kv_tile_count", "attn_tile_kind", "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attention",
+    "attn_fwd_schedule",
     "attn_hadamard_quant_fp8_noalloc", "lib_path", "EXPORTS",
 ]
 
@@ -34,7 +35,7 @@ lib_path = os.path.join(_HERE, "libattn.so")
 EXPORTS = (
     "attn_fwd", "attn_fwd_fp8", "attn_hadamard_quant_fp8", "attn_hadamard_quant_fp8_workspace_bytes",
     "attn_get_last_device_error", "attn_status_string", "attn_kv_tile_count", "attn_tile_kind",
-    "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attn_hadamard_quant_fp8_noalloc",
+    "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attn_hadamard_quant_fp8_noalloc", "attn_fwd_schedule",
 )
 
 if not os.path.exists(lib_path):
@@ -61,6 +62,8 @@ _lib.attn_kv_tile_count.argtypes = [_I] * 6
 _lib.attn_kv_tile_count.restype = _I
 _lib.attn_tile_kind.argtypes = [_I] * 7
 _lib.attn_tile_kind.restype = _I
+_lib.attn_fwd_schedule.argtypes = [_I]
+_lib.attn_fwd_schedule.restype = _I
 _lib.attn_debug_unsatisfied_wait.argtypes = [_LL, _vp]
 _lib.attn_debug_unsatisfied_wait.restype = _I
 _lib.attn_debug_exp2.argtypes = [_vp, _vp, _LL, _I, _vp]
@@ -144,6 +147,11 @@ def attn_kv_tile_count(row0, row1, Nq, Nk, bn, causal) -> int:
 
 def attn_tile_kind(row0, row1, kt, Nq, Nk, bn, causal) -> int:
     return int(_lib.attn_tile_kind(row0, row1, kt, Nq, Nk, bn, int(causal)))
+
+
+def attn_fwd_schedule(Nk) -> int:
+    """1 if attn_fwd runs the persistent kernel for Nk keys, 0 for one block per item."""
+    return int(_lib.attn_fwd_schedule(Nk))
 
 
 def attn_debug_unsatisfied_wait(limit_ns: int, stream=None, raise_on_error=True):

@@ -299,6 +299,8 @@ int attn_kv_tile_count(int row0, int row1, int Nq, int Nk, int bn, int causal) {
   return kv_tile_count(row0, row1, Nq, Nk, bn, causal != 0);
 }
 
+int attn_fwd_schedule(int Nk) { return Nk < 0 ? -1 : (Nk <= kPersistentMaxNk ? 1 : 0); }
+
 int attn_tile_kind(int row0, int row1, int kt, int Nq, int Nk, int bn, int causal) {
   if (row0 < 0 || row1 < row0 || kt < 0 || Nq < 0 || Nk < 0 || bn <= 0 || (causal != 0 && causal != 1)) return -1;
   return tile_kind(row0, row1, kt, Nq, Nk, bn, causal != 0);

@@ -174,6 +174,16 @@ int attn_kv_tile_count(int row0, int row1, int Nq, int Nk, int bn, int causal);
 int attn_tile_kind(int row0, int row1, int kt, int Nq, int Nk, int bn, int causal);
 
 /*
+ * Which kernel attn_fwd / attn_fwd_fp8 launch for a key range of Nk keys:
+ * 1 = the persistent kernel (one block per SM looping over the work items;
+ * used for short key ranges, whose items are short), 0 = one block per work
+ * item.  Both compute the same result.  Host-only; -1 if Nk < 0.  The page
+ * set describes one block per (batch, head, query block); the persistent
+ * schedule is this library's own.
+ */
+int attn_fwd_schedule(int Nk);
+
+/*
  * Debug hook for the failure path: launches one block that waits, with the
  * given limit in nanoseconds, on a device barrier nothing ever completes, so
  * the bounded wait runs out and records ATTN_ERR_DEVICE_TIMEOUT in the

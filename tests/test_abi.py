@@ -89,3 +89,9 @@ def test_debug_probe_rejects_bad_limits():
 def test_error_raises():
     with pytest.raises(ea.AttnError):
         ea.attn_fwd(FAKE, FAKE, FAKE, FAKE, None, 1, 3, 2, 8, 8, 128, 0, 0.1, 0, stream=0)
+
+
+def test_schedule_boundary():
+    # persistent kernel for key ranges up to 1024, one block per item above
+    assert ea.attn_fwd_schedule(-1) == -1
+    assert [ea.attn_fwd_schedule(n) for n in (0, 1, 1024, 1025, 8192)] == [1, 1, 1, 0, 0]
