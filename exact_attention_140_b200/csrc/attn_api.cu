@@ -240,18 +240,23 @@ int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, 
 // start for each.  Longer items run one block per item.
 constexpr int kPersistentMaxNk = 1024;
 
-template <int D, int BN, int NQT, int KST, int VST, bool FP8, int EMU, int SB = (NQT == 1 ? 2 : 1)>
+// PSEP: the persistent kernel gives P tensor-memory columns of its own
+// (where they fit: d = 64 with two query tiles uses all 512 columns).
+template <int D, int BN, int NQT, int KST, int VST, bool FP8, int EMU, bool PSEP = false,
+          int SB = (NQT == 1 ? 2 : 1)>
 int launch_causal(bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                   int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
                   DeviceState* st, cudaStream_t s) {
   const bool persist = Nk <= kPersistentMaxNk;
   if (causal) {
     using C = FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU, SB>;
-    return persist ? launch_fwd_persistent<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
+    using CP = FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU, SB, PSEP>;
+    return persist ? launch_fwd_persistent<CP>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
                    : launch_fwd<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
   }
   using C = FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU, SB>;
-  return persist ? launch_fwd_persistent<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
+  using CP = FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU, SB, PSEP>;
+  return persist ? launch_fwd_persistent<CP>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
                  : launch_fwd<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
 }
 
@@ -336,7 +341,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   const bool c = causal != 0;
   switch (d) {
     case 64:  // 3 of 8 exponentials in software: at d = 64 the exponential costs twice the tensor time
-      return launch_causal<64, 128, 2, 3, 3, false, 3>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
+      return launch_causal<64, 128, 2, 3, 3, false, 3, true>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
                                                        nullptr, nullptr, st, s);
     case 128:  // 2 of 8 exponentials in software
       return launch_causal<128, 128, 2, 2, 2, false, 2>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,

@@ -28,9 +28,13 @@ struct FwdParams {
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
 
 template <int D_, int BN_, int NQT_, int KST_, int VST_, bool CAUSAL_, bool FP8_, int EMU_ = 0,
-          int SB_ = (NQT_ == 1 ? 2 : 1)>
+          int SB_ = (NQT_ == 1 ? 2 : 1), bool PSEP_ = false>
 struct FwdCfg {
   static constexpr int D = D_, BN = BN_, NQT = NQT_, KST = KST_, VST = VST_;
+  // PSEP: P gets tensor-memory columns of its own instead of overwriting S,
+  // so Q K_{j+1}^T can be computed while the softmax of tile j still runs
+  // (persistent kernel only; needs a single score buffer per query tile)
+  static constexpr bool PSEP = PSEP_;
   // software exp2 share on full tiles: element pairs with (pair % 8) < EMU
   static constexpr int EMU = EMU_;
   static constexpr bool CAUSAL = CAUSAL_, FP8 = FP8_;
@@ -48,7 +52,9 @@ struct FwdCfg {
   static constexpr int QK_STEPS = D / KSTEP;
   static constexpr int PV_STEPS = BN / KSTEP;
   static constexpr int P_COLS = BN * ELEM / 4;
-  static constexpr int O_COL0 = NQT * SB * BN;
+  static constexpr int P_COL0 = NQT * SB * BN;  // P of tile t at P_COL0 + t * P_COLS (PSEP only)
+  static constexpr int O_COL0 = NQT * SB * BN + (PSEP ? NQT * P_COLS : 0);
+  static_assert(!PSEP || SB == 1, "separate P with one score buffer");
   static constexpr int TMEM_USED = O_COL0 + NQT * D;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   static_assert(TMEM_USED <= 512, "tensor memory has 512 columns");
@@ -67,7 +73,8 @@ struct FwdCfg {
   static constexpr int B_OFINAL = B_ODONE + NQT;
   static constexpr int B_OFREE = B_OFINAL + NQT;
   static constexpr int B_QEMPTY = B_OFREE + NQT;
-  static constexpr int B_DRAIN = B_QEMPTY + 1;
+  static constexpr int B_SFREE = B_QEMPTY + 1;  // S read out of tensor memory (PSEP)
+  static constexpr int B_DRAIN = B_SFREE + NQT * SB;
   static constexpr int NBAR = B_DRAIN + 1;
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr uint32_t OFF_Q = 0;
@@ -138,5 +145,11 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Wa
   return wait_bar_slow<ROLE>(bar, parity, c, site);
 }
 enum : int { kRoleSoftmax = 0, kRoleProducer = 1, kRoleMma = 2 };
+// Wait by a whole warp (every lane polls the same barrier); the result is made
+// warp-uniform so that the warp stays converged on the error path too.
+template <int ROLE>
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, const WaitCtx& c, uint32_t site) {
+  return __all_sync(0xffffffffu, wait_bar<ROLE>(bar, parity, c, site));
+}
 
 }  // namespace attn

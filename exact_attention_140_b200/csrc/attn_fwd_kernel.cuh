@@ -58,6 +58,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   constexpr int BM = Cfg::BM, BN = Cfg::BN, D = Cfg::D, NQT = Cfg::NQT, SB = Cfg::SB;
+  static_assert(!Cfg::PSEP, "P overwrites S in this kernel");
   constexpr int KST = Cfg::KST, VST = Cfg::VST;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
@@ -367,11 +368,13 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
   }
   if (warp == Cfg::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop (waits, counters, descriptors); one
+    // elected lane issues the tcgen05 instructions.
+    {
       bool ok = true;
 #pragma unroll
       for (int t = 0; t < NQT && ok; ++t)
-        if (n_kv[t] > 0) ok = wait_bar<kRoleMma>(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
+        if (n_kv[t] > 0) ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
       ptx::tc_fence_after();
       const uint32_t q_s = sbase + Cfg::OFF_Q, k_s = sbase + Cfg::OFF_K, v_s = sbase + Cfg::OFF_V;
       auto issue_qk = [&](int t, int j) {
@@ -385,13 +388,13 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
           const uint32_t ch = (uint32_t)kk / 4u, in = (uint32_t)kk % 4u;
           const uint64_t ad = ad0 + (uint64_t)((ch * Cfg::CH_Q + in * 32u) >> 4);
           const uint64_t bd = bd0 + (uint64_t)((ch * Cfg::CH_KV + in * 32u) >> 4);
-          ptx::mma_ss<Cfg::FP8>(d_t, ad, bd, Cfg::IDESC_QK, kk > 0 ? 1u : 0u);
+          ptx::warp_mma_ss<Cfg::FP8>(d_t, ad, bd, Cfg::IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        ptx::tc_commit(bar(Cfg::B_SFULL + t * SB + j % SB));
+        ptx::warp_commit(bar(Cfg::B_SFULL + t * SB + j % SB));
       };
       auto issue_pv = [&](int t, int jj) -> bool {
         const int si = t * SB + jj % SB;
-        if (!wait_bar<kRoleMma>(bar(Cfg::B_PFULL + si), (uint32_t)((jj / SB) & 1), wc, kSitePFull)) return false;
+        if (!wait_bar_warp<kRoleMma>(bar(Cfg::B_PFULL + si), (uint32_t)((jj / SB) & 1), wc, kSitePFull)) return false;
         ptx::tc_fence_after();
         const uint32_t d_t = tmem + (uint32_t)(Cfg::O_COL0 + t * D);
         const uint32_t a_t = tmem + (uint32_t)(si * BN);
@@ -399,10 +402,10 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < Cfg::PV_STEPS; ++kk) {
           const uint64_t bd = bd0 + (uint64_t)(((uint32_t)kk * Cfg::KSTEP * 128u) >> 4);
-          ptx::mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+          ptx::warp_mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
         }
-        ptx::tc_commit(bar(Cfg::B_ODONE + t));
-        if (jj == n_kv[t] - 1) ptx::tc_commit(bar(Cfg::B_OFINAL + t));
+        ptx::warp_commit(bar(Cfg::B_ODONE + t));
+        if (jj == n_kv[t] - 1) ptx::warp_commit(bar(Cfg::B_OFINAL + t));
         return true;
       };
       for (int j = 0; ok && j <= nmax; ++j) {
@@ -412,16 +415,16 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
           // they run under the softmax of key tile j-1; then the P V of
           // key tile j-1 as each tile's P is released
           if (has_k) {
-            ok = wait_bar<kRoleMma>(bar(Cfg::B_KFULL + j % KST), (uint32_t)((j / KST) & 1), wc, kSiteKFull);
+            ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_KFULL + j % KST), (uint32_t)((j / KST) & 1), wc, kSiteKFull);
             if (!ok) break;
             ptx::tc_fence_after();
 #pragma unroll
             for (int t = 0; t < NQT; ++t)
               if (j < n_kv[t]) issue_qk(t, j);
-            ptx::tc_commit(bar(Cfg::B_KEMPTY + j % KST));
+            ptx::warp_commit(bar(Cfg::B_KEMPTY + j % KST));
           }
           if (has_v) {
-            ok = wait_bar<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc,
+            ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc,
                                     kSiteVFull);
             if (!ok) break;
             ptx::tc_fence_after();
@@ -429,17 +432,17 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
             for (int t = 0; t < NQT && ok; ++t)
               if (j - 1 < n_kv[t]) ok = issue_pv(t, j - 1);
             if (!ok) break;
-            ptx::tc_commit(bar(Cfg::B_VEMPTY + (j - 1) % VST));
+            ptx::warp_commit(bar(Cfg::B_VEMPTY + (j - 1) % VST));
           }
         } else {
           // P overwrites S in place: PV(t, j-1) must be issued before
           // QK(t, j) reuses the buffer
           if (has_k) {
-            ok = wait_bar<kRoleMma>(bar(Cfg::B_KFULL + j % KST), (uint32_t)((j / KST) & 1), wc, kSiteKFull);
+            ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_KFULL + j % KST), (uint32_t)((j / KST) & 1), wc, kSiteKFull);
             if (!ok) break;
           }
           if (has_v) {
-            ok = wait_bar<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc,
+            ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc,
                                     kSiteVFull);
             if (!ok) break;
           }
@@ -450,13 +453,13 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
             if (ok && has_k && j < n_kv[t]) issue_qk(t, j);
           }
           if (!ok) break;
-          if (has_k) ptx::tc_commit(bar(Cfg::B_KEMPTY + j % KST));
-          if (has_v) ptx::tc_commit(bar(Cfg::B_VEMPTY + (j - 1) % VST));
+          if (has_k) ptx::warp_commit(bar(Cfg::B_KEMPTY + j % KST));
+          if (has_v) ptx::warp_commit(bar(Cfg::B_VEMPTY + (j - 1) % VST));
         }
       }
       // All issued MMAs must finish before tensor memory is freed.
-      ptx::tc_commit(bar(Cfg::B_DRAIN));
-      wait_bar<kRoleMma>(bar(Cfg::B_DRAIN), 0u, wc, kSiteDrain);
+      ptx::warp_commit(bar(Cfg::B_DRAIN));
+      wait_bar_warp<kRoleMma>(bar(Cfg::B_DRAIN), 0u, wc, kSiteDrain);
     }
   }
 

@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       ptx::mbar_init(bar(Cfg::B_OFREE + t), 128);
     }
     ptx::mbar_init(bar(Cfg::B_QEMPTY), 1);
+    for (int i = 0; i < NQT * SB; ++i) ptx::mbar_init(bar(Cfg::B_SFREE + i), 128);
     ptx::mbar_init(bar(Cfg::B_DRAIN), 1);
     *abort_flag = 0u;
     ptx::fence_mbar_init();
@@ -163,6 +164,11 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
           ptx::tmem_ld32(s_taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) ptx::tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+        if constexpr (Cfg::PSEP) {
+          // S is in registers: the next Q K^T of this tile may overwrite it
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bar(Cfg::B_SFREE + si));
+        }
         float m_blk;
         if (partial) {
           float mx = -INFINITY;
@@ -198,6 +204,20 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         }
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         const bool resc_any = __any_sync(0xffffffffu, resc);
+        if constexpr (Cfg::PSEP) {
+          // P has one buffer per tile: the previous P V (product scount - 1)
+          // must have read it.  Product scount cannot have completed (its P is
+          // not written yet) and product scount - 2 was waited for one tile
+          // earlier, so the parity test is unambiguous.
+          if (scount > 0) {
+            ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_ODONE + t), (uint32_t)((scount - 1) & 1), wc, kSiteODone);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            ptx::tc_fence_after();
+          }
+        }
+        const uint32_t p_taddr =
+            Cfg::PSEP ? tmem + lane_off + (uint32_t)(Cfg::P_COL0 + t * Cfg::P_COLS) : s_taddr;
         // ---- exponentiate 32 columns at a time; each chunk's packed P is
         // stored at once (over score columns already read), so the registers
         // of a chunk die before the next chunk is processed
@@ -244,9 +264,9 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
               }
             }
             if constexpr (Cfg::FP8)
-              ptx::tmem_st8(s_taddr + (uint32_t)(PW * ch), pk);
+              ptx::tmem_st8(p_taddr + (uint32_t)(PW * ch), pk);
             else
-              ptx::tmem_st16(s_taddr + (uint32_t)(PW * ch), pk);
+              ptx::tmem_st16(p_taddr + (uint32_t)(PW * ch), pk);
             if (ch == BN / 64 - 1 && !resc_any) {
               // the first half of P is in TMEM: its P V can start while the
               // second half is exponentiated (a warp that must rescale O
@@ -430,15 +450,24 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
   }
   if (warp == Cfg::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop (waits, counters, descriptors); one
+    // elected lane issues the tcgen05 instructions.
+    {
       bool ok = true;
       const uint32_t q_s = sbase + Cfg::OFF_Q, k_s = sbase + Cfg::OFF_K, v_s = sbase + Cfg::OFF_V;
       int kc = 0, vc = 0;                  // K / V ring slots consumed
       int scount[NQT], pcount[NQT], qcount[NQT], ouse[NQT];
 #pragma unroll
       for (int t = 0; t < NQT; ++t) scount[t] = pcount[t] = qcount[t] = ouse[t] = 0;
-      auto issue_qk = [&](int t, int kslot) {
+      auto issue_qk = [&](int t, int kslot) -> bool {
         const int buf = scount[t] % SB;
+        if constexpr (Cfg::PSEP) {
+          // the softmax must have read the previous S of this buffer
+          if (scount[t] > 0 && !wait_bar_warp<kRoleMma>(bar(Cfg::B_SFREE + t * SB + buf),
+                                                   (uint32_t)((scount[t] - 1) & 1), wc, kSiteSFull))
+            return false;
+          ptx::tc_fence_after();
+        }
         const uint32_t d_t = tmem + (uint32_t)((t * SB + buf) * BN);
         // descriptors advance by 32 bytes (>> 4 = 2) per K step inside a
         // 128-byte chunk and by one chunk (CH_Q / CH_KV bytes) after four
@@ -449,17 +478,18 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
           const uint32_t ch = (uint32_t)kk / 4u, in = (uint32_t)kk % 4u;
           const uint64_t ad = ad0 + (uint64_t)((ch * Cfg::CH_Q + in * 32u) >> 4);
           const uint64_t bd = bd0 + (uint64_t)((ch * Cfg::CH_KV + in * 32u) >> 4);
-          ptx::mma_ss<Cfg::FP8>(d_t, ad, bd, Cfg::IDESC_QK, kk > 0 ? 1u : 0u);
+          ptx::warp_mma_ss<Cfg::FP8>(d_t, ad, bd, Cfg::IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        ptx::tc_commit(bar(Cfg::B_SFULL + t * SB + buf));
+        ptx::warp_commit(bar(Cfg::B_SFULL + t * SB + buf));
         ++scount[t];
+        return true;
       };
       // P V of key tile jj of the current item; jj == 0 starts a new output
       auto issue_pv = [&](int t, int jj, int vslot, bool last) -> bool {
         if (jj == 0) {
           // the previous item's output of this tile must have been read out
           if (ouse[t] > 0 &&
-              !wait_bar<kRoleMma>(bar(Cfg::B_OFREE + t), (uint32_t)((ouse[t] - 1) & 1), wc, kSiteODone))
+              !wait_bar_warp<kRoleMma>(bar(Cfg::B_OFREE + t), (uint32_t)((ouse[t] - 1) & 1), wc, kSiteODone))
             return false;
           ++ouse[t];
         }
@@ -467,23 +497,23 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         const int si = t * SB + buf;
         const uint32_t ph = (uint32_t)((pcount[t] / SB) & 1);
         const uint32_t d_t = tmem + (uint32_t)(Cfg::O_COL0 + t * D);
-        const uint32_t a_t = tmem + (uint32_t)(si * BN);
+        const uint32_t a_t = tmem + (uint32_t)(Cfg::PSEP ? Cfg::P_COL0 + t * Cfg::P_COLS : si * BN);
         const uint64_t bd0 = ptx::sdesc_sw128(v_s + vslot * Cfg::KV_BYTES, Cfg::CH_KV, 1024u);
         // the first half of the keys as soon as their P is written, the rest
         // when the whole P is
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          if (!wait_bar<kRoleMma>(bar((half == 0 ? Cfg::B_PHALF : Cfg::B_PFULL) + si), ph, wc, kSitePFull))
+          if (!wait_bar_warp<kRoleMma>(bar((half == 0 ? Cfg::B_PHALF : Cfg::B_PFULL) + si), ph, wc, kSitePFull))
             return false;
           ptx::tc_fence_after();
 #pragma unroll
           for (int kk = half * Cfg::PV_STEPS / 2; kk < (half + 1) * Cfg::PV_STEPS / 2; ++kk) {
             const uint64_t bd = bd0 + (uint64_t)(((uint32_t)kk * Cfg::KSTEP * 128u) >> 4);
-            ptx::mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+            ptx::warp_mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        ptx::tc_commit(bar(Cfg::B_ODONE + t));
-        if (last) ptx::tc_commit(bar(Cfg::B_OFINAL + t));
+        ptx::warp_commit(bar(Cfg::B_ODONE + t));
+        if (last) ptx::warp_commit(bar(Cfg::B_OFINAL + t));
         ++pcount[t];
         return true;
       };
@@ -496,7 +526,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
 #pragma unroll
         for (int t = 0; t < NQT && ok; ++t)
           if (n_kv[t] > 0) {
-            ok = wait_bar<kRoleMma>(bar(Cfg::B_QFULL + t), (uint32_t)(qcount[t] & 1), wc, kSiteQ);
+            ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_QFULL + t), (uint32_t)(qcount[t] & 1), wc, kSiteQ);
             ++qcount[t];
           }
         if (!ok) break;
@@ -509,62 +539,69 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
             // they run under the softmax of key tile j-1; then the P V of
             // key tile j-1 as each tile's P is released
             if (has_k) {
-              ok = wait_bar<kRoleMma>(bar(Cfg::B_KFULL + ks), (uint32_t)((kc / KST) & 1), wc, kSiteKFull);
+              ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_KFULL + ks), (uint32_t)((kc / KST) & 1), wc, kSiteKFull);
               if (!ok) break;
               ptx::tc_fence_after();
 #pragma unroll
               for (int t = 0; t < NQT; ++t)
-                if (j < n_kv[t]) issue_qk(t, ks);
-              ptx::tc_commit(bar(Cfg::B_KEMPTY + ks));
+                if (j < n_kv[t]) issue_qk(t, ks);  // no wait inside: SB == 2 excludes PSEP
+              ptx::warp_commit(bar(Cfg::B_KEMPTY + ks));
               ++kc;
             }
             if (has_v) {
-              ok = wait_bar<kRoleMma>(bar(Cfg::B_VFULL + vs), (uint32_t)((vc / VST) & 1), wc, kSiteVFull);
+              ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_VFULL + vs), (uint32_t)((vc / VST) & 1), wc, kSiteVFull);
               if (!ok) break;
               ptx::tc_fence_after();
 #pragma unroll
               for (int t = 0; t < NQT && ok; ++t)
                 if (j - 1 < n_kv[t]) ok = issue_pv(t, j - 1, vs, j == n_kv[t]);
               if (!ok) break;
-              ptx::tc_commit(bar(Cfg::B_VEMPTY + vs));
+              ptx::warp_commit(bar(Cfg::B_VEMPTY + vs));
               ++vc;
             }
           } else {
             // P overwrites S in place: PV(t, j-1) must be issued before
-            // QK(t, j) reuses the buffer
+            // QK(t, j) reuses the buffer.  With a separate P buffer the order
+            // turns round: QK(t, j) needs only S(t, j-1) read out, which the
+            // softmax signals early, and PV(t, j-1) waits for the whole P.
             if (has_k) {
-              ok = wait_bar<kRoleMma>(bar(Cfg::B_KFULL + ks), (uint32_t)((kc / KST) & 1), wc, kSiteKFull);
+              ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_KFULL + ks), (uint32_t)((kc / KST) & 1), wc, kSiteKFull);
               if (!ok) break;
             }
             if (has_v) {
-              ok = wait_bar<kRoleMma>(bar(Cfg::B_VFULL + vs), (uint32_t)((vc / VST) & 1), wc, kSiteVFull);
+              ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_VFULL + vs), (uint32_t)((vc / VST) & 1), wc, kSiteVFull);
               if (!ok) break;
             }
             ptx::tc_fence_after();
 #pragma unroll
             for (int t = 0; t < NQT && ok; ++t) {
-              if (has_v && j - 1 < n_kv[t]) ok = issue_pv(t, j - 1, vs, j == n_kv[t]);
-              if (ok && has_k && j < n_kv[t]) issue_qk(t, ks);
+              if constexpr (Cfg::PSEP) {
+                if (has_k && j < n_kv[t]) ok = issue_qk(t, ks);
+                if (ok && has_v && j - 1 < n_kv[t]) ok = issue_pv(t, j - 1, vs, j == n_kv[t]);
+              } else {
+                if (has_v && j - 1 < n_kv[t]) ok = issue_pv(t, j - 1, vs, j == n_kv[t]);
+                if (ok && has_k && j < n_kv[t]) ok = issue_qk(t, ks);
+              }
             }
             if (!ok) break;
             if (has_k) {
-              ptx::tc_commit(bar(Cfg::B_KEMPTY + ks));
+              ptx::warp_commit(bar(Cfg::B_KEMPTY + ks));
               ++kc;
             }
             if (has_v) {
-              ptx::tc_commit(bar(Cfg::B_VEMPTY + vs));
+              ptx::warp_commit(bar(Cfg::B_VEMPTY + vs));
               ++vc;
             }
           }
           // after the item's last Q K^T: Q smem is free once it completes,
           // so the next item's Q can load under this item's last P V
-          if (j == nmax - 1) ptx::tc_commit(bar(Cfg::B_QEMPTY));
+          if (j == nmax - 1) ptx::warp_commit(bar(Cfg::B_QEMPTY));
         }
-        if (nmax == 0) ptx::tc_commit(bar(Cfg::B_QEMPTY));
+        if (nmax == 0) ptx::warp_commit(bar(Cfg::B_QEMPTY));
       }
       // All issued MMAs must finish before tensor memory is freed.
-      ptx::tc_commit(bar(Cfg::B_DRAIN));
-      wait_bar<kRoleMma>(bar(Cfg::B_DRAIN), 0u, wc, kSiteDrain);
+      ptx::warp_commit(bar(Cfg::B_DRAIN));
+      wait_bar_warp<kRoleMma>(bar(Cfg::B_DRAIN), 0u, wc, kSiteDrain);
     }
   }
 

@@ -126,6 +126,36 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
   }
 }
 
+// Warp-level issue: the whole (converged) warp runs the issuing loop and one
+// lane, chosen by elect.sync, issues each tcgen05 instruction.  elect.sync
+// elects the same lane every time for the same member mask, so the commits
+// (which track the MMAs of the lane that issues them) see every MMA.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+template <bool kFP8>
+__device__ __forceinline__ void warp_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  if (elect_one()) mma_ss<kFP8>(d_tmem, a_desc, b_desc, idesc, accumulate);
+  __syncwarp();
+}
+template <bool kFP8>
+__device__ __forceinline__ void warp_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  if (elect_one()) mma_ts<kFP8>(d_tmem, a_tmem, b_desc, idesc, accumulate);
+  __syncwarp();
+}
+__device__ __forceinline__ void warp_commit(uint32_t bar) {
+  if (elect_one()) tc_commit(bar);
+  __syncwarp();
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled tile (tcgen05
 // format): start address, leading- and stride-dimension byte offsets (all in
 // 16-byte units), the fixed version field (bit 46 = 1) and layout type 2
