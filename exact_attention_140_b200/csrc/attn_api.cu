@@ -240,9 +240,11 @@ int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, 
 // start for each.  Longer items run one block per item.
 constexpr int kPersistentMaxNk = 1024;
 
+// EMU / EMU_P: share of the softmax exponentials computed in software (out of
+// 8 element pairs) in the one-block-per-item and the persistent kernel.
 // PSEP: the persistent kernel gives P tensor-memory columns of its own
 // (where they fit: d = 64 with two query tiles uses all 512 columns).
-template <int D, int BN, int NQT, int KST, int VST, bool FP8, int EMU, bool PSEP = false,
+template <int D, int BN, int NQT, int KST, int VST, bool FP8, int EMU, int EMU_P, bool PSEP = false,
           int SB = (NQT == 1 ? 2 : 1)>
 int launch_causal(bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                   int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
@@ -250,12 +252,12 @@ int launch_causal(bool causal, const void* q, const void* k, const void* v, void
   const bool persist = Nk <= kPersistentMaxNk;
   if (causal) {
     using C = FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU, SB>;
-    using CP = FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU, SB, PSEP>;
+    using CP = FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU_P, SB, PSEP>;
     return persist ? launch_fwd_persistent<CP>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
                    : launch_fwd<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
   }
   using C = FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU, SB>;
-  using CP = FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU, SB, PSEP>;
+  using CP = FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU_P, SB, PSEP>;
   return persist ? launch_fwd_persistent<CP>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
                  : launch_fwd<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
 }
@@ -340,13 +342,13 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
   const bool c = causal != 0;
   switch (d) {
-    case 64:  // 3 of 8 exponentials in software: at d = 64 the exponential costs twice the tensor time
-      return launch_causal<64, 128, 2, 3, 3, false, 3, true>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
+    case 64:  // software exponentials: 3 of 8 on long key ranges, none on short ones (measured)
+      return launch_causal<64, 128, 2, 3, 3, false, 3, 0, true>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
                                                        nullptr, nullptr, st, s);
-    case 128:  // 2 of 8 exponentials in software
-      return launch_causal<128, 128, 2, 2, 2, false, 2>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
+    case 128:  // 2 of 8 exponentials in software on long key ranges, none on short ones
+      return launch_causal<128, 128, 2, 2, 2, false, 2, 0>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
                                                         nullptr, nullptr, st, s);
-    default: return launch_causal<256, 64, 1, 2, 2, false, 0>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
+    default: return launch_causal<256, 64, 1, 2, 2, false, 0, 0>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
                                                              nullptr, nullptr, st, s);
   }
 }
@@ -364,7 +366,7 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float*
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
-  return launch_causal<128, 128, 2, 3, 3, true, 3>(causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, scale,
+  return launch_causal<128, 128, 2, 3, 3, true, 3, 3>(causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, scale,
                                                     descale_q, descale_k, descale_v, st, s);
 }
 
