@@ -229,7 +229,8 @@ int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, 
   if ((rc = encode_qkv<Cfg>(&tq, &tk, &tv, q, k, v, B, Hq, Hkv, Nq, Nk)) != ATTN_OK) return rc;
   FwdParams p;
   if (!fill_params<Cfg>(&p, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st)) return ATTN_ERR_UNSUPPORTED;
-  const int nblk = p.n_items < st->num_sms ? p.n_items : st->num_sms;
+  const int nstreams = (p.n_items + Cfg::NS - 1) / Cfg::NS;  // blocks that find work
+  const int nblk = nstreams < st->num_sms ? nstreams : st->num_sms;
   attn_fwd_persistent_kernel<Cfg><<<dim3((unsigned)nblk), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -240,26 +241,29 @@ int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, 
 // start for each.  Longer items run one block per item.
 constexpr int kPersistentMaxNk = 1024;
 
-// EMU / EMU_P: share of the softmax exponentials computed in software (out of
-// 8 element pairs) in the one-block-per-item and the persistent kernel.
-// PSEP: the persistent kernel gives P tensor-memory columns of its own
-// (where they fit: d = 64 with two query tiles uses all 512 columns).
-template <int D, int BN, int NQT, int KST, int VST, bool FP8, int EMU, int EMU_P, bool PSEP = false,
-          int SB = (NQT == 1 ? 2 : 1)>
-int launch_causal(bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
-                  DeviceState* st, cudaStream_t s) {
+// Kernel configurations, FwdCfg<D, BN, NQT, KST, VST, CAUSAL, FP8, EMU, SB,
+// PSEP, NS>: per head size a long-range one (one block per item) and a
+// short-range one (persistent).  EMU is the share of softmax exponentials
+// computed in software (out of 8 element pairs), chosen by measurement.
+//   d = 64 short: two independent streams of one 128-row query tile each; P
+//   in columns of its own (S 128 + P 64 + O 64 = 256 columns per stream).
+template <bool C> using CfgD64 = FwdCfg<64, 128, 2, 3, 3, C, false, 3>;
+template <bool C> using CfgD64Short = FwdCfg<64, 128, 1, 3, 3, C, false, 2, 1, true, 2>;
+template <bool C> using CfgD128 = FwdCfg<128, 128, 2, 2, 2, C, false, 2>;
+template <bool C> using CfgD128Short = FwdCfg<128, 128, 2, 2, 2, C, false, 0>;
+template <bool C> using CfgD256 = FwdCfg<256, 64, 1, 2, 2, C, false, 0>;
+template <bool C> using CfgFP8 = FwdCfg<128, 128, 2, 3, 3, C, true, 3>;
+
+template <template <bool> class Long, template <bool> class Short>
+int launch_sched(bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                 int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
+                 DeviceState* st, cudaStream_t s) {
   const bool persist = Nk <= kPersistentMaxNk;
-  if (causal) {
-    using C = FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU, SB>;
-    using CP = FwdCfg<D, BN, NQT, KST, VST, true, FP8, EMU_P, SB, PSEP>;
-    return persist ? launch_fwd_persistent<CP>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
-                   : launch_fwd<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
-  }
-  using C = FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU, SB>;
-  using CP = FwdCfg<D, BN, NQT, KST, VST, false, FP8, EMU_P, SB, PSEP>;
-  return persist ? launch_fwd_persistent<CP>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
-                 : launch_fwd<C>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
+  if (causal)
+    return persist ? launch_fwd_persistent<Short<true>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
+                   : launch_fwd<Long<true>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
+  return persist ? launch_fwd_persistent<Short<false>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
+                 : launch_fwd<Long<false>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
 }
 
 int check_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
@@ -342,14 +346,15 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
   const bool c = causal != 0;
   switch (d) {
-    case 64:  // software exponentials: 3 of 8 on long key ranges, none on short ones (measured)
-      return launch_causal<64, 128, 2, 3, 3, false, 3, 0, true>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
-                                                       nullptr, nullptr, st, s);
-    case 128:  // 2 of 8 exponentials in software on long key ranges, none on short ones
-      return launch_causal<128, 128, 2, 2, 2, false, 2, 0>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
-                                                        nullptr, nullptr, st, s);
-    default: return launch_causal<256, 64, 1, 2, 2, false, 0, 0>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr,
-                                                             nullptr, nullptr, st, s);
+    case 64:
+      return launch_sched<CfgD64, CfgD64Short>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr, nullptr,
+                                               st, s);
+    case 128:
+      return launch_sched<CfgD128, CfgD128Short>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr,
+                                                 nullptr, st, s);
+    default:
+      return launch_sched<CfgD256, CfgD256>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr, nullptr,
+                                            st, s);
   }
 }
 
@@ -366,8 +371,8 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float*
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
-  return launch_causal<128, 128, 2, 3, 3, true, 3, 3>(causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, scale,
-                                                    descale_q, descale_k, descale_v, st, s);
+  return launch_sched<CfgFP8, CfgFP8>(causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, scale, descale_q, descale_k,
+                                      descale_v, st, s);
 }
 
 long long attn_hadamard_quant_fp8_workspace_bytes(void) { return 256; }

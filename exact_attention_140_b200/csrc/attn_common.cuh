@@ -28,9 +28,14 @@ struct FwdParams {
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
 
 template <int D_, int BN_, int NQT_, int KST_, int VST_, bool CAUSAL_, bool FP8_, int EMU_ = 0,
-          int SB_ = (NQT_ == 1 ? 2 : 1), bool PSEP_ = false>
+          int SB_ = (NQT_ == 1 ? 2 : 1), bool PSEP_ = false, int NS_ = 1>
 struct FwdCfg {
   static constexpr int D = D_, BN = BN_, NQT = NQT_, KST = KST_, VST = VST_;
+  // NS: independent streams per block (persistent kernel): each has its own
+  // softmax warpgroup(s), TMA and MMA warps, K/V rings, barriers and tensor
+  // memory columns, and takes its own work items
+  static constexpr int NS = NS_;
+  static_assert(NS == 1 || (NS == 2 && NQT == 1), "two streams of one query tile each");
   // PSEP: P gets tensor-memory columns of its own instead of overwriting S,
   // so Q K_{j+1}^T can be computed while the softmax of tile j still runs
   // (persistent kernel only; needs a single score buffer per query tile)
@@ -55,9 +60,10 @@ struct FwdCfg {
   static constexpr int P_COL0 = NQT * SB * BN;  // P of tile t at P_COL0 + t * P_COLS (PSEP only)
   static constexpr int O_COL0 = NQT * SB * BN + (PSEP ? NQT * P_COLS : 0);
   static_assert(!PSEP || SB == 1, "separate P with one score buffer");
-  static constexpr int TMEM_USED = O_COL0 + NQT * D;
-  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
-  static_assert(TMEM_USED <= 512, "tensor memory has 512 columns");
+  static constexpr int TMEM_USED = O_COL0 + NQT * D;  // columns of one stream
+  static constexpr int TMEM_ALL = NS * TMEM_USED;
+  static constexpr int TMEM_COLS = TMEM_ALL <= 128 ? 128 : (TMEM_ALL <= 256 ? 256 : 512);
+  static_assert(TMEM_ALL <= 512, "tensor memory has 512 columns");
   static_assert(D % 64 == 0 && NCH >= 1, "head size");
   static_assert(BN % 32 == 0 && BN <= 256, "key tile");
   // barriers
@@ -76,19 +82,23 @@ struct FwdCfg {
   static constexpr int B_SFREE = B_QEMPTY + 1;  // S read out of tensor memory (PSEP)
   static constexpr int B_DRAIN = B_SFREE + NQT * SB;
   static constexpr int NBAR = B_DRAIN + 1;
-  // shared memory (offsets from a 1024-byte aligned base)
+  // shared memory (offsets from a 1024-byte aligned base; stream s adds
+  // s * STREAM_BYTES to the tile offsets and s * NBAR to barrier indices)
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + NQT * QT_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + VST * KV_BYTES;
-  static constexpr uint32_t OFF_SLOT = OFF_BAR + NBAR * 8;
+  static constexpr uint32_t STREAM_BYTES = OFF_V + VST * KV_BYTES;
+  static constexpr uint32_t OFF_BAR = NS * STREAM_BYTES;
+  static constexpr uint32_t OFF_SLOT = OFF_BAR + NS * NBAR * 8;
   static constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
   static constexpr uint32_t SMEM_BYTES = OFF_ABORT + 4 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per block");
-  // warps: softmax warpgroups, then one warpgroup holding the TMA warp, the
-  // MMA warp and two idle warps (a whole warpgroup, so that registers can be
-  // moved to the softmax warpgroups with setmaxnreg)
-  static constexpr int SM_WARPS = 4 * NQT;
+  // warps: softmax warpgroups (stream s owns warps 4*NQT*s ..), then one
+  // warpgroup holding the TMA and MMA warps of each stream (TMA warp of stream
+  // s = SM_WARPS + 2s, its MMA warp the next one) and, with one stream, two
+  // idle warps (a whole warpgroup, so that registers can be moved to the
+  // softmax warpgroups with setmaxnreg)
+  static constexpr int SM_WARPS = 4 * NQT * NS;
   static constexpr int TMA_WARP = SM_WARPS;
   static constexpr int MMA_WARP = SM_WARPS + 1;
   static constexpr int NTHREADS = 32 * (SM_WARPS + 4);
@@ -96,7 +106,7 @@ struct FwdCfg {
   // 64512; softmax warpgroups get 224, the control warpgroup keeps 56:
   // 2*128*224 + 128*56 = 64512)
   static constexpr int REG_LAUNCH = 65536 / NTHREADS >= 255 ? 255 : (65536 / NTHREADS) / 8 * 8;
-  static constexpr bool SPLIT_REGS = NQT == 2;
+  static constexpr bool SPLIT_REGS = NQT * NS == 2;
   static constexpr int REG_SOFTMAX = 200, REG_CONTROL = 104;
   static_assert(!SPLIT_REGS || 2 * 128 * REG_SOFTMAX + 128 * REG_CONTROL <= NTHREADS * REG_LAUNCH,
                 "register split exceeds the launch allocation");
@@ -116,6 +126,13 @@ struct WaitCtx {
   unsigned long long timeout_ns;
 };
 
+// Warp roles, for the per-role instantiation of the polling loop.  A producer
+// that shares its scheduler with busy softmax warps (two streams per block)
+// polls with a short sleep between rounds (kRoleProducerBackoff): it runs
+// stages ahead, so the added wake-up latency costs nothing, and the issue
+// slots go to the softmax warps.
+enum : int { kRoleSoftmax = 0, kRoleProducer = 1, kRoleMma = 2, kRoleProducerBackoff = 3 };
+
 // Bounded mbarrier wait: true when the phase with `parity` has completed;
 // false after the time limit (recording the site in the error word and
 // raising the block's abort flag) or when another role already aborted.
@@ -131,6 +148,7 @@ __device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, const 
     for (int i = 0; i < 16; ++i)
       if (ptx::mbar_try_wait(bar, parity)) return true;
     if (*c.abort) return false;
+    if constexpr (ROLE == kRoleProducerBackoff) __nanosleep(64);
     if (ptx::globaltimer() - t0 > c.timeout_ns) {
       *c.abort = 1u;
       const uint32_t blk = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
@@ -144,7 +162,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Wa
   if (ptx::mbar_try_wait(bar, parity)) return true;
   return wait_bar_slow<ROLE>(bar, parity, c, site);
 }
-enum : int { kRoleSoftmax = 0, kRoleProducer = 1, kRoleMma = 2 };
+
 // Wait by a whole warp (every lane polls the same barrier); the result is made
 // warp-uniform so that the warp stays converged on the error path too.
 template <int ROLE>

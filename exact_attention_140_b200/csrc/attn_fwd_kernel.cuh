@@ -14,8 +14,9 @@
 //   warp 4*NQT          TMA producer: Q tiles once, then K_j and V_j through
 //                       KST / VST-stage shared-memory rings (section 2: the
 //                       next block is fetched while the current one computes);
-//   warp 4*NQT+1        MMA issuer: one thread issues every tcgen05.mma;
-//                       also allocates and frees tensor memory;
+//   warp 4*NQT+1        MMA issuer: the warp runs the issue loop and one
+//                       elected lane issues every tcgen05.mma; it also
+//                       allocates and frees tensor memory;
 //   warps 4*NQT+2, +3   idle (they complete the control warpgroup, whose
 //                       registers are handed to the softmax warpgroups).
 //
@@ -424,8 +425,8 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
             ptx::warp_commit(bar(Cfg::B_KEMPTY + j % KST));
           }
           if (has_v) {
-            ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc,
-                                    kSiteVFull);
+            ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1),
+                                         wc, kSiteVFull);
             if (!ok) break;
             ptx::tc_fence_after();
 #pragma unroll
@@ -442,8 +443,8 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
             if (!ok) break;
           }
           if (has_v) {
-            ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1), wc,
-                                    kSiteVFull);
+            ok = wait_bar_warp<kRoleMma>(bar(Cfg::B_VFULL + (j - 1) % VST), (uint32_t)(((j - 1) / VST) & 1),
+                                         wc, kSiteVFull);
             if (!ok) break;
           }
           ptx::tc_fence_after();

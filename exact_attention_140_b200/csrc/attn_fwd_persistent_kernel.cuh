@@ -2,13 +2,13 @@
 // attention forward, for short key ranges.
 //
 // It computes the same thing as attn_fwd_kernel (same tiles, warp roles,
-// tensor-memory layout, online softmax with lazy rescaling and epilogue; see
-// that file), but a grid of one block per SM loops over the work items
-// (batch, query head, query block) instead of launching one block per item.
-// With short key ranges an item is only a few key tiles long and the fixed
-// costs around it -- block start, tensor-memory allocation, the first Q and
-// K/V loads, the epilogue's read-out of O -- are a large share of its time;
-// here they overlap with the neighbouring items:
+// online softmax with lazy rescaling and epilogue; see that file), but a grid
+// of one block per SM loops over the work items (batch, query head, query
+// block) instead of launching one block per item.  With short key ranges an
+// item is only a few key tiles long and the fixed costs around it -- block
+// start, tensor-memory allocation, the first Q and K/V loads, the epilogue's
+// read-out of O -- are a large share of its time; here they overlap with the
+// neighbouring items:
 //   * the producer issues the next item's first K/V tile while the current
 //     item is still computing, and its Q tile as soon as the last Q K^T of
 //     the current item has completed (barrier q_empty);
@@ -19,6 +19,19 @@
 //     first half of the keys starts while the second half is exponentiated.
 // Ring slots and barrier phases are counted across items, so the pipeline
 // never drains between them.
+//
+// Two layouts of the block:
+//   * NS = 1: NQT query tiles of one item share the K/V stream (as in
+//     attn_fwd_kernel);
+//   * NS = 2 (d = 64): two independent streams, each with one softmax
+//     warpgroup, its own TMA and MMA warps (the four warps of the control
+//     warpgroup), K/V rings, barriers and 256 tensor-memory columns, taking
+//     128-row work items of their own.  The streams do not wait for each
+//     other at item boundaries, which with causal masks (query tiles of one
+//     item differ in length) left a tile idle for about a step per item.
+// PSEP (d = 64) gives P columns of its own (S 128 + P 64 + O 64 per tile), so
+// Q K_{j+1}^T runs during the softmax of tile j; the softmax signals s_free
+// once S is in registers and waits for the previous P V before writing P.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -33,12 +46,12 @@
 namespace attn {
 
 // Work items are (batch, query head, query block).  The grid is persistent
-// (one block per SM); block c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... of an
-// order sorted longest-first (for causal masks), so long and short items pair
-// up.  Head-major order keeps the query blocks of one head on the GPU at the
-// same time (their K/V tiles are shared through L2).
-__device__ __forceinline__ int item_at(int k, int G, int T) {
-  const int c = (int)blockIdx.x;
+// (one block per SM, NS streams per block); stream c of G takes items c,
+// 2G-1-c, 2G+c, 4G-1-c, ... of an order sorted longest-first (for causal
+// masks), so long and short items pair up.  Head-major order keeps the query
+// blocks of one head on the GPU at the same time (their K/V tiles are shared
+// through L2).
+__device__ __forceinline__ int item_at(int k, int G, int T, int c) {
   const long long pos = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
   return pos < T ? (int)pos : -1;
 }
@@ -68,12 +81,22 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
   const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
   const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - raw_u32);
-  auto bar = [&](int i) -> uint32_t { return sbase + Cfg::OFF_BAR + 8u * (uint32_t)i; };
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sgen + Cfg::OFF_ABORT);
   const WaitCtx wc{abort_flag, p.err, p.timeout_ns};
-  const int G = (int)gridDim.x, T = p.n_items;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // role and stream of this warp
+  const int cw = warp - Cfg::SM_WARPS;  // index within the control warpgroup
+  const bool is_tma = cw >= 0 && cw < 2 * Cfg::NS && (cw & 1) == 0;
+  const bool is_mma = cw >= 0 && cw < 2 * Cfg::NS && (cw & 1) == 1;
+  const int s = warp < Cfg::SM_WARPS ? warp / (4 * NQT) : ((is_tma || is_mma) ? (cw >> 1) : 0);
+  auto bar_s = [&](int ss, int i) -> uint32_t {
+    return sbase + Cfg::OFF_BAR + 8u * (uint32_t)(ss * Cfg::NBAR + i);
+  };
+  auto bar = [&](int i) -> uint32_t { return bar_s(s, i); };
+  const uint32_t sstream = sbase + (uint32_t)s * Cfg::STREAM_BYTES;  // Q/K/V tiles of this stream
+  const int G = (int)gridDim.x * Cfg::NS, T = p.n_items;
+  const int c = (int)blockIdx.x * Cfg::NS + s;  // this stream's index in the grid
   // key tiles the query tiles of an item visit (0 = none)
   auto plan = [&](const Item& it, int (&n_kv)[NQT]) -> int {
     const int q0 = it.qb * BM * NQT;
@@ -87,32 +110,34 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
   };
 
   if (threadIdx.x == 0) {
-    for (int t = 0; t < NQT; ++t) ptx::mbar_init(bar(Cfg::B_QFULL + t), 1);
+    for (int ss = 0; ss < Cfg::NS; ++ss) {
+    for (int t = 0; t < NQT; ++t) ptx::mbar_init(bar_s(ss, Cfg::B_QFULL + t), 1);
     for (int s = 0; s < KST; ++s) {
-      ptx::mbar_init(bar(Cfg::B_KFULL + s), 1);
-      ptx::mbar_init(bar(Cfg::B_KEMPTY + s), 1);
+      ptx::mbar_init(bar_s(ss, Cfg::B_KFULL + s), 1);
+      ptx::mbar_init(bar_s(ss, Cfg::B_KEMPTY + s), 1);
     }
     for (int s = 0; s < VST; ++s) {
-      ptx::mbar_init(bar(Cfg::B_VFULL + s), 1);
-      ptx::mbar_init(bar(Cfg::B_VEMPTY + s), 1);
+      ptx::mbar_init(bar_s(ss, Cfg::B_VFULL + s), 1);
+      ptx::mbar_init(bar_s(ss, Cfg::B_VEMPTY + s), 1);
     }
     for (int i = 0; i < NQT * SB; ++i) {
-      ptx::mbar_init(bar(Cfg::B_SFULL + i), 1);
-      ptx::mbar_init(bar(Cfg::B_PFULL + i), 128);
-      ptx::mbar_init(bar(Cfg::B_PHALF + i), 128);
+      ptx::mbar_init(bar_s(ss, Cfg::B_SFULL + i), 1);
+      ptx::mbar_init(bar_s(ss, Cfg::B_PFULL + i), 128);
+      ptx::mbar_init(bar_s(ss, Cfg::B_PHALF + i), 128);
     }
     for (int t = 0; t < NQT; ++t) {
-      ptx::mbar_init(bar(Cfg::B_ODONE + t), 1);
-      ptx::mbar_init(bar(Cfg::B_OFINAL + t), 1);
-      ptx::mbar_init(bar(Cfg::B_OFREE + t), 128);
+      ptx::mbar_init(bar_s(ss, Cfg::B_ODONE + t), 1);
+      ptx::mbar_init(bar_s(ss, Cfg::B_OFINAL + t), 1);
+      ptx::mbar_init(bar_s(ss, Cfg::B_OFREE + t), 128);
     }
-    ptx::mbar_init(bar(Cfg::B_QEMPTY), 1);
-    for (int i = 0; i < NQT * SB; ++i) ptx::mbar_init(bar(Cfg::B_SFREE + i), 128);
-    ptx::mbar_init(bar(Cfg::B_DRAIN), 1);
+    ptx::mbar_init(bar_s(ss, Cfg::B_QEMPTY), 1);
+    for (int i = 0; i < NQT * SB; ++i) ptx::mbar_init(bar_s(ss, Cfg::B_SFREE + i), 128);
+    ptx::mbar_init(bar_s(ss, Cfg::B_DRAIN), 1);
+    }
     *abort_flag = 0u;
     ptx::fence_mbar_init();
   }
-  if (warp == Cfg::TMA_WARP && lane == 0) {
+  if (is_tma && lane == 0) {
     ptx::prefetch_tmap(&tmQ);
     ptx::prefetch_tmap(&tmK);
     ptx::prefetch_tmap(&tmV);
@@ -125,20 +150,21 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sgen + Cfg::OFF_SLOT);
+  const uint32_t tmem_s = tmem + (uint32_t)(s * Cfg::TMEM_USED);  // this stream's columns
 
   if (warp < Cfg::SM_WARPS) {
     // ------------------------------------------------------------ softmax
     if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_inc<Cfg::REG_SOFTMAX>();
-    const int t = warp >> 2, wq = warp & 3;
+    const int t = (warp >> 2) % NQT, wq = warp & 3;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t o_taddr = tmem + lane_off + (uint32_t)(Cfg::O_COL0 + t * D);
+    const uint32_t o_taddr = tmem_s + lane_off + (uint32_t)(Cfg::O_COL0 + t * D);
     float sl2 = p.sl2;
     if constexpr (Cfg::FP8) sl2 *= __ldg(p.dq) * __ldg(p.dk);
     int scount = 0;       // score buffers of this query tile consumed so far (= P V products issued before)
     int finals = 0;       // items whose output this tile has written
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int item = item_at(k, G, T);
+      const int item = item_at(k, G, T, c);
       if (item < 0) break;
       const Item it = decode_item(item, p);
       int n_kv[NQT];
@@ -154,7 +180,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint32_t s_taddr = tmem + lane_off + (uint32_t)(si * BN);
+        const uint32_t s_taddr = tmem_s + lane_off + (uint32_t)(si * BN);
         const bool partial = tile_kind(row0, row0 + BM, j, p.Nq, p.Nk, BN, Cfg::CAUSAL) == kTilePartial;
         const int nvis = vend - j * BN;  // visible keys of this tile (masks partial tiles)
         // ---- one read of the whole score row (one TMEM load latency per tile)
@@ -217,7 +243,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
           }
         }
         const uint32_t p_taddr =
-            Cfg::PSEP ? tmem + lane_off + (uint32_t)(Cfg::P_COL0 + t * Cfg::P_COLS) : s_taddr;
+            Cfg::PSEP ? tmem_s + lane_off + (uint32_t)(Cfg::P_COL0 + t * Cfg::P_COLS) : s_taddr;
         // ---- exponentiate 32 columns at a time; each chunk's packed P is
         // stored at once (over score columns already read), so the registers
         // of a chunk die before the next chunk is processed
@@ -356,8 +382,9 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         p.lse[((long long)ie.b * p.Hq + ie.h) * p.Nq + row] = lse;
       }
     }
-  } else if (warp == Cfg::TMA_WARP) {
+  } else if (is_tma) {
     // ------------------------------------------------------------ producer
+    constexpr int kProducerRole = Cfg::NS > 1 ? kRoleProducerBackoff : kRoleProducer;
     if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_dec<Cfg::REG_CONTROL>();
     if (lane == 0) {
       int k_issued[KST], v_issued[VST], q_issued[NQT];
@@ -370,7 +397,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       int kc = 0, vc = 0;  // loads issued into the K and V rings
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int item = item_at(k, G, T);
+        const int item = item_at(k, G, T, c);
         if (item < 0) break;
         const Item it = decode_item(item, p);
         int n_kv[NQT];
@@ -380,28 +407,28 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         auto load_kv = [&](int j) -> bool {
           const int ks = kc % KST;
           if (kc >= KST &&
-              !wait_bar<kRoleProducer>(bar(Cfg::B_KEMPTY + ks), (uint32_t)(((kc / KST) - 1) & 1), wc, kSiteKEmpty))
+              !wait_bar<kProducerRole>(bar(Cfg::B_KEMPTY + ks), (uint32_t)(((kc / KST) - 1) & 1), wc, kSiteKEmpty))
             return false;
           {
             const uint32_t fb = bar(Cfg::B_KFULL + ks);
             ptx::mbar_arrive_expect_tx(fb, Cfg::KV_BYTES);
 #pragma unroll
             for (int c = 0; c < Cfg::NCH; ++c)
-              ptx::tma_load_4d(sbase + Cfg::OFF_K + ks * Cfg::KV_BYTES + c * Cfg::CH_KV, &tmK, fb, c * Cfg::BOXE, kh,
+              ptx::tma_load_4d(sstream + Cfg::OFF_K + ks * Cfg::KV_BYTES + c * Cfg::CH_KV, &tmK, fb, c * Cfg::BOXE, kh,
                                j * BN, it.b);
             ++k_issued[ks];
             ++kc;
           }
           const int vs = vc % VST;
           if (vc >= VST &&
-              !wait_bar<kRoleProducer>(bar(Cfg::B_VEMPTY + vs), (uint32_t)(((vc / VST) - 1) & 1), wc, kSiteVEmpty))
+              !wait_bar<kProducerRole>(bar(Cfg::B_VEMPTY + vs), (uint32_t)(((vc / VST) - 1) & 1), wc, kSiteVEmpty))
             return false;
           {
             const uint32_t fb = bar(Cfg::B_VFULL + vs);
             ptx::mbar_arrive_expect_tx(fb, Cfg::KV_BYTES);
 #pragma unroll
             for (int c = 0; c < Cfg::NCH; ++c)
-              ptx::tma_load_4d(sbase + Cfg::OFF_V + vs * Cfg::KV_BYTES + c * Cfg::CH_KV, &tmV, fb, c * Cfg::BOXE, kh,
+              ptx::tma_load_4d(sstream + Cfg::OFF_V + vs * Cfg::KV_BYTES + c * Cfg::CH_KV, &tmV, fb, c * Cfg::BOXE, kh,
                                j * BN, it.b);
             ++v_issued[vs];
             ++vc;
@@ -412,7 +439,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         // is in flight while the previous item finishes
         if (nmax > 0 && !load_kv(0)) break;
         // Q smem is free once the previous item's last Q K^T has completed
-        if (k > 0 && !wait_bar<kRoleProducer>(bar(Cfg::B_QEMPTY), (uint32_t)((k - 1) & 1), wc, kSiteQ)) break;
+        if (k > 0 && !wait_bar<kProducerRole>(bar(Cfg::B_QEMPTY), (uint32_t)((k - 1) & 1), wc, kSiteQ)) break;
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
           if (n_kv[t] == 0) continue;
@@ -420,7 +447,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
           ptx::mbar_arrive_expect_tx(fb, Cfg::QT_BYTES);
 #pragma unroll
           for (int c = 0; c < Cfg::NCH; ++c)
-            ptx::tma_load_4d(sbase + Cfg::OFF_Q + t * Cfg::QT_BYTES + c * Cfg::CH_Q, &tmQ, fb, c * Cfg::BOXE, it.h,
+            ptx::tma_load_4d(sstream + Cfg::OFF_Q + t * Cfg::QT_BYTES + c * Cfg::CH_Q, &tmQ, fb, c * Cfg::BOXE, it.h,
                              q0 + t * BM, it.b);
           ++q_issued[t];
         }
@@ -435,26 +462,26 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
 #pragma unroll
       for (int t = 0; t < NQT; ++t)
         if (q_issued[t] > 0)
-          wait_bar<kRoleProducer>(bar(Cfg::B_QFULL + t), (uint32_t)((q_issued[t] - 1) & 1), wc, kSiteQ);
+          wait_bar<kProducerRole>(bar(Cfg::B_QFULL + t), (uint32_t)((q_issued[t] - 1) & 1), wc, kSiteQ);
 #pragma unroll
       for (int s = 0; s < KST; ++s)
         if (k_issued[s] > 0)
-          wait_bar<kRoleProducer>(bar(Cfg::B_KFULL + s), (uint32_t)((k_issued[s] - 1) & 1), wc, kSiteKFull);
+          wait_bar<kProducerRole>(bar(Cfg::B_KFULL + s), (uint32_t)((k_issued[s] - 1) & 1), wc, kSiteKFull);
 #pragma unroll
       for (int s = 0; s < VST; ++s)
         if (v_issued[s] > 0)
-          wait_bar<kRoleProducer>(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
+          wait_bar<kProducerRole>(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
     }
   } else {
     if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_dec<Cfg::REG_CONTROL>();
   }
-  if (warp == Cfg::MMA_WARP) {
+  if (is_mma) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs this loop (waits, counters, descriptors); one
     // elected lane issues the tcgen05 instructions.
     {
       bool ok = true;
-      const uint32_t q_s = sbase + Cfg::OFF_Q, k_s = sbase + Cfg::OFF_K, v_s = sbase + Cfg::OFF_V;
+      const uint32_t q_s = sstream + Cfg::OFF_Q, k_s = sstream + Cfg::OFF_K, v_s = sstream + Cfg::OFF_V;
       int kc = 0, vc = 0;                  // K / V ring slots consumed
       int scount[NQT], pcount[NQT], qcount[NQT], ouse[NQT];
 #pragma unroll
@@ -464,11 +491,11 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         if constexpr (Cfg::PSEP) {
           // the softmax must have read the previous S of this buffer
           if (scount[t] > 0 && !wait_bar_warp<kRoleMma>(bar(Cfg::B_SFREE + t * SB + buf),
-                                                   (uint32_t)((scount[t] - 1) & 1), wc, kSiteSFull))
+                                                        (uint32_t)((scount[t] - 1) & 1), wc, kSiteSFull))
             return false;
           ptx::tc_fence_after();
         }
-        const uint32_t d_t = tmem + (uint32_t)((t * SB + buf) * BN);
+        const uint32_t d_t = tmem_s + (uint32_t)((t * SB + buf) * BN);
         // descriptors advance by 32 bytes (>> 4 = 2) per K step inside a
         // 128-byte chunk and by one chunk (CH_Q / CH_KV bytes) after four
         const uint64_t ad0 = ptx::sdesc_sw128(q_s + t * Cfg::QT_BYTES, 16u, 1024u);
@@ -496,8 +523,8 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         const int buf = pcount[t] % SB;
         const int si = t * SB + buf;
         const uint32_t ph = (uint32_t)((pcount[t] / SB) & 1);
-        const uint32_t d_t = tmem + (uint32_t)(Cfg::O_COL0 + t * D);
-        const uint32_t a_t = tmem + (uint32_t)(Cfg::PSEP ? Cfg::P_COL0 + t * Cfg::P_COLS : si * BN);
+        const uint32_t d_t = tmem_s + (uint32_t)(Cfg::O_COL0 + t * D);
+        const uint32_t a_t = tmem_s + (uint32_t)(Cfg::PSEP ? Cfg::P_COL0 + t * Cfg::P_COLS : si * BN);
         const uint64_t bd0 = ptx::sdesc_sw128(v_s + vslot * Cfg::KV_BYTES, Cfg::CH_KV, 1024u);
         // the first half of the keys as soon as their P is written, the rest
         // when the whole P is
@@ -518,7 +545,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         return true;
       };
       for (int k = 0; ok; ++k) {
-        const int item = item_at(k, G, T);
+        const int item = item_at(k, G, T, c);
         if (item < 0) break;
         const Item it = decode_item(item, p);
         int n_kv[NQT];
