@@ -79,4 +79,5 @@ def compare(o, lse, o_ref, lse_ref, tol=BF16_TOL):
         d = np.abs(lse[~empty] - lse_ref[~empty])
         if d.size:
             assert d.max() <= tol["lse"], f"max |dLSE| = {d.max():.3g}"
-    return float(err.max()), float(err.mean())
+        return float(err.max()), float(err.mean()), float(d.max()) if d.size else 0.0
+    return float(err.max()), float(err.mean()), None

@@ -47,4 +47,5 @@ def test_fullsize_sampled_rows(name):
     o_ref, lse_ref = oracle.attn_fwd_rows(gen.bf16_bits_to_f64(qb), gen.bf16_bits_to_f64(kb),
                                           gen.bf16_bits_to_f64(vb), causal, scale, rows)
     b, h, i = rows // (Hq * N), (rows // N) % Hq, rows % N
-    compare(o[b, i, h, :], lse[b, h, i], o_ref, lse_ref)
+    emax, emean, dlse = compare(o[b, i, h, :], lse[b, h, i], o_ref, lse_ref)
+    print(f"{name}: {rows.size} rows, max |dO| {emax:.3e}, mean |dO| {emean:.3e}, max |dLSE| {dlse:.3e}")
