@@ -56,6 +56,11 @@ def lib():
                                          [ctypes.c_double, _I, ctypes.c_double,
                                           ctypes.POINTER(_LL)])
         L.oracle_attn_online.restype = _I
+        L.oracle_attn_fwd_window.argtypes = ([_dp, _dp, _dp, _dp, _dp] + [_I] * 7 +
+                                             [ctypes.c_double, _LL, _LL])
+        L.oracle_attn_fwd_window.restype = _I
+        L.oracle_combine.argtypes = [_dp, _dp, _I, _LL, _I, _dp, _dp]
+        L.oracle_combine.restype = _I
         L.oracle_attn_bruteforce.argtypes = [_dp, _dp, _dp, _dp, _dp] + [_I] * 7 + [ctypes.c_double]
         L.oracle_attn_bruteforce.restype = _I
         L.oracle_mask.argtypes = [_I, _I, _I, _u8]
@@ -100,6 +105,44 @@ def attn_fwd(q, k, v, causal: bool, scale: float):
     if rc:
         raise ValueError(f"oracle_attn_fwd failed ({rc})")
     return o, lse
+
+
+def attn_fwd_window(q, k, v, causal: bool, scale: float, k0: int, k1: int):
+    """The definition over the keys [k0, k1) only (causal rule in absolute key
+    indices): one window's partial result.  Returns O [B,Nq,Hq,d], LSE [B,Hq,Nq];
+    rows with no allowed key in the window get O = 0, LSE = -inf."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Hq, d, Nk = _shape(q, k, k.shape[2])
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq, Nq))
+    rc = lib().oracle_attn_fwd_window(q, k, v, o, lse, B, Hq, k.shape[2], Nq, Nk, d, int(causal), scale,
+                                      int(k0), int(k1))
+    if rc:
+        raise ValueError(f"oracle_attn_fwd_window failed ({rc})")
+    return o, lse
+
+
+def combine(o_parts, lse_parts):
+    """Merge S partial results: o_parts [S, ..., d] and lse_parts [S, ...] with
+    matching row order.  Returns O [..., d] and LSE [...]."""
+    o_parts, lse_parts = _f64(o_parts), _f64(lse_parts)
+    S, d = o_parts.shape[0], o_parts.shape[-1]
+    R = int(np.prod(o_parts.shape[1:-1]))
+    if lse_parts.shape[0] != S or int(np.prod(lse_parts.shape[1:])) != R:
+        raise ValueError("o_parts / lse_parts shapes do not match")
+    o = np.zeros(o_parts.shape[1:])
+    lse = np.zeros(lse_parts.shape[1:])
+    if lib().oracle_combine(o_parts, lse_parts, S, R, d, o, lse):
+        raise ValueError("oracle_combine failed")
+    return o, lse
+
+
+def combine_bnhd(o_parts, lse_parts):
+    """combine() for the library's partial layouts: o_parts [S,B,Nq,Hq,d],
+    lse_parts [S,B,Hq,Nq].  Returns O [B,Nq,Hq,d] and LSE [B,Hq,Nq]."""
+    lse_rows = np.ascontiguousarray(np.transpose(_f64(lse_parts), (0, 1, 3, 2)))  # [S,B,Nq,Hq]
+    o, lse = combine(o_parts, lse_rows)
+    return o, np.ascontiguousarray(np.transpose(lse, (0, 2, 1)))
 
 
 def attn_fwd_rows(q, k, v, causal: bool, scale: float, rows):

@@ -34,6 +34,14 @@
  *                          with an optional lazy threshold tau on the max
  *                          update (page "FlashAttention-4震撼发布", the new
  *                          online softmax that skips most output rescalings).
+ *   oracle_attn_fwd_window the definition over the keys [k0, k1) only (the
+ *                          mask rule unchanged, in absolute key indices): the
+ *                          partial result of one key window of split-KV.
+ *   oracle_combine         merge of partial results over disjoint key windows,
+ *                          O = sum_s e^(LSE_s - LSE) O_s with LSE = ln sum_s
+ *                          e^(LSE_s): the rescaling step of the online softmax
+ *                          (page "FlashAttention (SV)", section "Online-beräkning
+ *                          av Softmax") applied to whole windows.
  *   oracle_attn_bruteforce long-double, materialised S, p_j = 1/sum_k e^(s_k-s_j):
  *                          a different algebra, for tiny inputs.
  *   oracle_hadamard        M = diag(s) H_d / sqrt(d) (Sylvester H_d), the random
@@ -58,16 +66,17 @@ static int allowed(long long i, long long j, long long Nq, long long Nk, int cau
     return j <= i + (Nk - Nq);
 }
 
-/* One output row: query (b, h, i).  q_row points at Q[b,i,h,:]. */
+/* One output row: query (b, h, i) over the keys [j_lo, j_hi) (the whole
+ * range is [0, Nk)).  q_row points at Q[b,i,h,:]. */
 static void attend_row(const double *q_row, const double *k, const double *v,
                        int b, int h, long long i, int Hq, int Hkv, int Nq, int Nk,
-                       int d, int causal, double scale, double *s, double *o_row,
-                       double *lse_out)
+                       int d, int causal, double scale, long long j_lo, long long j_hi,
+                       double *s, double *o_row, double *lse_out)
 {
     const int kh = h / (Hq / Hkv);
     double m = -INFINITY;
     int any = 0;
-    for (long long j = 0; j < Nk; ++j) {
+    for (long long j = j_lo; j < j_hi; ++j) {
         if (!allowed(i, j, Nq, Nk, causal)) continue;
         const double *k_row = k + (((long long)b * Nk + j) * Hkv + kh) * d;
         double dot = 0.0;
@@ -79,7 +88,7 @@ static void attend_row(const double *q_row, const double *k, const double *v,
     for (int c = 0; c < d; ++c) o_row[c] = 0.0;
     if (!any) { *lse_out = -INFINITY; return; }
     double l = 0.0;
-    for (long long j = 0; j < Nk; ++j) {
+    for (long long j = j_lo; j < j_hi; ++j) {
         if (!allowed(i, j, Nq, Nk, causal)) continue;
         const double w = exp(s[j] - m);
         const double *v_row = v + (((long long)b * Nk + j) * Hkv + kh) * d;
@@ -110,13 +119,81 @@ int oracle_attn_fwd(const double *q, const double *k, const double *v, double *o
                 const int h = (int)((r / Nq) % Hq);
                 const long long i = r % Nq;
                 const long long qo = (((long long)b * Nq + i) * Hq + h) * d;
-                attend_row(q + qo, k, v, b, h, i, Hq, Hkv, Nq, Nk, d, causal, scale, s,
+                attend_row(q + qo, k, v, b, h, i, Hq, Hkv, Nq, Nk, d, causal, scale, 0, Nk, s,
                            o + qo, lse + r);
             }
             free(s);
         }
     }
     return err;
+}
+
+/* The definition restricted to the keys [k0, k1) (clipped to [0, Nk)); the
+ * causal rule keeps its absolute form j <= i + (Nk - Nq).  Rows with no
+ * allowed key in the window get O = 0, LSE = -inf. */
+int oracle_attn_fwd_window(const double *q, const double *k, const double *v, double *o,
+                           double *lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                           int causal, double scale, long long k0, long long k1)
+{
+    if (Hkv <= 0 || Hq % Hkv) return 1;
+    if (k0 < 0) k0 = 0;
+    if (k1 > Nk) k1 = Nk;
+    const long long rows = (long long)B * Hq * Nq;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+        if (!s) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long long r = 0; r < rows; ++r) {
+                const int b = (int)(r / ((long long)Hq * Nq));
+                const int h = (int)((r / Nq) % Hq);
+                const long long i = r % Nq;
+                const long long qo = (((long long)b * Nq + i) * Hq + h) * d;
+                attend_row(q + qo, k, v, b, h, i, Hq, Hkv, Nq, Nk, d, causal, scale, k0, k1, s,
+                           o + qo, lse + r);
+            }
+            free(s);
+        }
+    }
+    return err;
+}
+
+/* Merge S partial results of R rows: o_parts[s*R*d + r*d + c], lse_parts[s*R + r]
+ * (natural log; -inf marks a window with no allowed key).  Writes o[r*d + c],
+ * lse[r]: LSE = ln sum_s exp(LSE_s), O = sum_s exp(LSE_s - LSE) O_s, computed
+ * with the largest LSE_s factored out; a row with every LSE_s = -inf gets
+ * O = 0, LSE = -inf. */
+int oracle_combine(const double *o_parts, const double *lse_parts, int S, long long R, int d,
+                   double *o, double *lse)
+{
+    if (S < 1 || R < 0 || d < 1) return 1;
+    for (long long r = 0; r < R; ++r) {
+        double m = -INFINITY;
+        for (int s = 0; s < S; ++s)
+            if (lse_parts[(long long)s * R + r] > m) m = lse_parts[(long long)s * R + r];
+        double *o_row = o + r * d;
+        for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+        if (m == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double wsum = 0.0;
+        for (int s = 0; s < S; ++s) {
+            const double ls = lse_parts[(long long)s * R + r];
+            if (ls == -INFINITY) continue;
+            const double w = exp(ls - m);
+            const double *src = o_parts + ((long long)s * R + r) * d;
+            wsum += w;
+            for (int c = 0; c < d; ++c) o_row[c] += w * src[c];
+        }
+        for (int c = 0; c < d; ++c) o_row[c] /= wsum;
+        lse[r] = m + log(wsum);
+    }
+    return 0;
 }
 
 /* rows[n] = flattened (b*Hq + h)*Nq + i; outputs o[n*d + c], lse[n]. */
@@ -146,7 +223,7 @@ int oracle_attn_fwd_rows(const double *q, const double *k, const double *v, doub
                 const int h = (int)((r / Nq) % Hq);
                 const long long i = r % Nq;
                 const long long qo = (((long long)b * Nq + i) * Hq + h) * d;
-                attend_row(q + qo, k, v, b, h, i, Hq, Hkv, Nq, Nk, d, causal, scale, s,
+                attend_row(q + qo, k, v, b, h, i, Hq, Hkv, Nq, Nk, d, causal, scale, 0, Nk, s,
                            o + n * d, lse + n);
             }
             free(s);
