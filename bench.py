@@ -48,6 +48,9 @@ def workloads():
         "mqa": dict(B=4, Hq=32, Hkv=1, N=4096, d=128, causal=True, dtype="bf16"),
         "d256": dict(B=2, Hq=8, Hkv=8, N=4096, d=256, causal=False, dtype="bf16"),
         "fp8": dict(B=4, Hq=16, Hkv=16, N=8192, d=128, causal=False, dtype="fp8"),
+        # decode-shaped (16 query rows against 32K keys), split-KV + combine;
+        # HBM-bound: the roofline is the K/V read
+        "decode": dict(B=4, Hq=32, Hkv=8, N=32768, Nq=16, d=128, causal=False, dtype="bf16", split=True),
     }
     for n in (512, 1024, 2048, 4096, 8192, 16384):
         for c in (False, True):
@@ -55,13 +58,19 @@ def workloads():
     return w
 
 
+def n_query(cfg) -> int:
+    """Query rows per head (N unless the workload sets Nq); N is the key count."""
+    return cfg.get("Nq", cfg["N"])
+
+
 def flops(cfg) -> float:
-    f = 4.0 * cfg["B"] * cfg["Hq"] * cfg["N"] * cfg["N"] * cfg["d"]
+    f = 4.0 * cfg["B"] * cfg["Hq"] * n_query(cfg) * cfg["N"] * cfg["d"]
     return f / 2 if cfg["causal"] else f
 
 
 def describe(name, cfg):
-    return (f"{name}: B={cfg['B']} Hq={cfg['Hq']} Hkv={cfg['Hkv']} N={cfg['N']} d={cfg['d']} "
+    n = f"N={cfg['N']}" if n_query(cfg) == cfg["N"] else f"Nq={n_query(cfg)} Nk={cfg['N']}"
+    return (f"{name}: B={cfg['B']} Hq={cfg['Hq']} Hkv={cfg['Hkv']} {n} d={cfg['d']} "
             f"{'causal' if cfg['causal'] else 'non-causal'} {cfg['dtype']}")
 
 
@@ -128,12 +137,13 @@ class ClockSampler:
 
 def make_inputs(cfg, seed=gen.BASE_SEED):
     outl = cfg["dtype"] == "fp8"
-    return gen.qkv_bf16(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["N"], cfg["N"], cfg["d"], seed=seed, outliers=outl)
+    return gen.qkv_bf16(cfg["B"], cfg["Hq"], cfg["Hkv"], n_query(cfg), cfg["N"], cfg["d"], seed=seed, outliers=outl)
 
 
 def _row_flops(cfg, rows):
-    i = rows % cfg["N"]
-    keys = np.minimum(cfg["N"], i + 1) if cfg["causal"] else np.full(rows.shape, cfg["N"])
+    nq, nk = n_query(cfg), cfg["N"]
+    i = rows % nq
+    keys = np.clip(i + (nk - nq) + 1, 0, nk) if cfg["causal"] else np.full(rows.shape, nk)
     return float(np.sum(4.0 * cfg["d"] * keys))
 
 
@@ -142,8 +152,8 @@ def oracle_sample(cfg, qb, kb, vb, target_s: float, n_rows: int | None = None, s
     keys).  With n_rows None the sample is grown until one run takes about
     target_s.  Returns (TFLOP/s, description, seconds, n_rows)."""
     import oracle
-    B, Hq, N, d = cfg["B"], cfg["Hq"], cfg["N"], cfg["d"]
-    total_rows = B * Hq * N
+    B, Hq, d = cfg["B"], cfg["Hq"], cfg["d"]
+    total_rows = B * Hq * n_query(cfg)
     q, k, v = gen.bf16_bits_to_f64(qb), gen.bf16_bits_to_f64(kb), gen.bf16_bits_to_f64(vb)
     rng = np.random.default_rng(seed)
     n = min(total_rows, n_rows or 256)
@@ -211,14 +221,15 @@ def run_ours(args, cfg, name):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     B, Hq, Hkv, N, d, causal = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["N"], cfg["d"], cfg["causal"]
+    Nq = n_query(cfg)
     scale = 1.0 / math.sqrt(d)
     fp8 = cfg["dtype"] == "fp8"
 
     qb, kb, vb = make_inputs(cfg, seed=gen.BASE_SEED + 1000 * rank)
     host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (qb, kb, vb)]
     q, k, v = (h.to(dev) for h in host)
-    o = torch.empty((B, N, Hq, d), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    o = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
     o_host = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
     lse_host = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -241,9 +252,17 @@ def run_ours(args, cfg, name):
             ea.attn_fwd_fp8(q8, k8, v8, o, lse, B, Hq, Hkv, N, N, d, causal, scale, desc.data_ptr(),
                             desc.data_ptr() + 4, desc.data_ptr() + 8, stream)
         launches_per_step = 7  # 3 x (amax + quantise) + attention
+    elif cfg.get("split"):
+        ws_bytes = ea.attn_splitkv_workspace_bytes(B, Hq, Nq, N, d, 0)
+        ws_split = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+
+        def step(qq, kk, vv):
+            ea.attn_fwd_splitkv(qq, kk, vv, o, lse, B, Hq, Hkv, Nq, N, d, causal, scale, 0, ws_split, ws_bytes,
+                                stream)
+        launches_per_step = 2 if ws_bytes > 0 else 1  # windows' attention + combine
     else:
         def step(qq, kk, vv):
-            ea.attn_fwd(qq, kk, vv, o, lse, B, Hq, Hkv, N, N, d, causal, scale, ea.ATTN_BF16, stream)
+            ea.attn_fwd(qq, kk, vv, o, lse, B, Hq, Hkv, Nq, N, d, causal, scale, ea.ATTN_BF16, stream)
         launches_per_step = 1
 
     for _ in range(max(3, args.warmup)):
@@ -331,6 +350,18 @@ def run_ours(args, cfg, name):
     achieved = f / kern_avg_s / 1e12
     peak = peaks["bf16"] * (2.0 if fp8 else 1.0)
     traffic = traffic_bytes(name)
+    if cfg.get("split"):
+        # HBM-bound: algorithmic bytes = Q + K + V read once, O + LSE written once
+        alg_bytes = float(sum(x.numel() * x.element_size() for x in (q, k, v, o, lse)))
+        roofline = {"bound": "hbm", "achieved": alg_bytes / kern_avg_s / 1e9, "peak": peaks["hbm"], "unit": "GB/s",
+                    "frac": alg_bytes / kern_avg_s / 1e9 / peaks["hbm"], "traffic": traffic,
+                    "peak_source": f"{peaks['src']} hbm copy", "kernel": "attn_fwd_kernel (key windows) + combine",
+                    "algorithmic_bytes": alg_bytes}
+    else:
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": traffic,
+                    "peak_source": f"{peaks['src']} {'bf16 x2 (fp8 nominal ratio)' if fp8 else 'bf16'}",
+                    "kernel": "attn_fwd_persistent_kernel" if ea.attn_fwd_schedule(N) == 1 else "attn_fwd_kernel"}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -339,10 +370,7 @@ def run_ours(args, cfg, name):
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "flushed between steps (256 MB write)",
                    "pct_of_peak": round(100.0 * value / world / peak, 2)},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"{peaks['src']} {'bf16 x2 (fp8 nominal ratio)' if fp8 else 'bf16'}",
-                     "kernel": "attn_fwd_persistent_kernel" if ea.attn_fwd_schedule(N) == 1 else "attn_fwd_kernel"},
+        "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in host)),
                 "d2h_bytes_per_step": int(o.numel() * o.element_size() + lse.numel() * lse.element_size())},

@@ -36,6 +36,8 @@ EXPORTS = (
     "attn_fwd", "attn_fwd_fp8", "attn_hadamard_quant_fp8", "attn_hadamard_quant_fp8_workspace_bytes",
     "attn_get_last_device_error", "attn_status_string", "attn_kv_tile_count", "attn_tile_kind",
     "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attn_hadamard_quant_fp8_noalloc", "attn_fwd_schedule",
+    "attn_fwd_splitkv", "attn_splitkv_workspace_bytes", "attn_combine", "attn_kv_tile_count_window",
+    "attn_tile_kind_window",
 )
 
 if not os.path.exists(lib_path):
@@ -68,6 +70,16 @@ _lib.attn_debug_unsatisfied_wait.argtypes = [_LL, _vp]
 _lib.attn_debug_unsatisfied_wait.restype = _I
 _lib.attn_debug_exp2.argtypes = [_vp, _vp, _LL, _I, _vp]
 _lib.attn_debug_exp2.restype = _I
+_lib.attn_splitkv_workspace_bytes.argtypes = [_I] * 6
+_lib.attn_splitkv_workspace_bytes.restype = _LL
+_lib.attn_fwd_splitkv.argtypes = [_vp] * 5 + [_I] * 7 + [_F, _I, _vp, _LL, _vp]
+_lib.attn_fwd_splitkv.restype = _I
+_lib.attn_combine.argtypes = [_vp, _vp] + [_I] * 5 + [_vp, _vp, _vp]
+_lib.attn_combine.restype = _I
+_lib.attn_kv_tile_count_window.argtypes = [_I] * 7
+_lib.attn_kv_tile_count_window.restype = _I
+_lib.attn_tile_kind_window.argtypes = [_I] * 8
+_lib.attn_tile_kind_window.restype = _I
 
 
 class AttnError(RuntimeError):
@@ -110,6 +122,23 @@ def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype=ATTN_B
     return _check(rc, "attn_fwd", raise_on_error)
 
 
+def attn_splitkv_workspace_bytes(B, Hq, Nq, Nk, d, n_splits=0) -> int:
+    return int(_lib.attn_splitkv_workspace_bytes(B, Hq, Nq, Nk, d, n_splits))
+
+
+def attn_fwd_splitkv(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, n_splits, workspace, workspace_bytes,
+                     stream=None, raise_on_error=True):
+    rc = _lib.attn_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, int(causal),
+                               float(scale), int(n_splits), _ptr(workspace), int(workspace_bytes), _stream(stream))
+    return _check(rc, "attn_fwd_splitkv", raise_on_error)
+
+
+def attn_combine(o_parts, lse_parts, n_splits, B, Hq, Nq, d, o, lse, stream=None, raise_on_error=True):
+    rc = _lib.attn_combine(_ptr(o_parts), _ptr(lse_parts), n_splits, B, Hq, Nq, d, _ptr(o), _ptr(lse),
+                           _stream(stream))
+    return _check(rc, "attn_combine", raise_on_error)
+
+
 def attn_fwd_fp8(q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, descale_q, descale_k, descale_v,
                  stream=None, raise_on_error=True):
     rc = _lib.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, int(causal),
@@ -147,6 +176,14 @@ def attn_kv_tile_count(row0, row1, Nq, Nk, bn, causal) -> int:
 
 def attn_tile_kind(row0, row1, kt, Nq, Nk, bn, causal) -> int:
     return int(_lib.attn_tile_kind(row0, row1, kt, Nq, Nk, bn, int(causal)))
+
+
+def attn_kv_tile_count_window(row0, row1, Nq, Nk, shift, bn, causal) -> int:
+    return int(_lib.attn_kv_tile_count_window(row0, row1, Nq, Nk, shift, bn, int(causal)))
+
+
+def attn_tile_kind_window(row0, row1, kt, Nq, Nk, shift, bn, causal) -> int:
+    return int(_lib.attn_tile_kind_window(row0, row1, kt, Nq, Nk, shift, bn, int(causal)))
 
 
 def attn_fwd_schedule(Nk) -> int:

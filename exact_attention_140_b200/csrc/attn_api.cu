@@ -12,6 +12,7 @@
 #include "attn.h"
 #include "attn_fwd_kernel.cuh"
 #include "attn_fwd_persistent_kernel.cuh"
+#include "combine.cuh"
 #include "fp8_prep.cuh"
 #include "tiles.h"
 
@@ -29,6 +30,7 @@ static __device__ __align__(256) unsigned int g_noalloc_scratch[kNoAllocScratchB
 __device__ float g_unit_descale = 1.0f;  // descale used when attn_fwd is given e4m3 inputs
 
 constexpr int kMaxDevices = 64;
+constexpr int kMaxSplits = 1024;  // key windows of one split-KV call
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
 
 struct DeviceState {
@@ -174,6 +176,10 @@ bool fill_params(FwdParams* p, void* o, float* lse, int B, int Hq, int Hkv, int 
   p->dv = dv;
   p->err = st->err;
   p->timeout_ns = timeout_ns();
+  p->n_splits = 1;
+  p->kv_chunk = Nk;
+  p->o_part = nullptr;
+  p->lse_part = nullptr;
   return true;
 }
 
@@ -233,6 +239,82 @@ int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, 
   const int nblk = nstreams < st->num_sms ? nstreams : st->num_sms;
   attn_fwd_persistent_kernel<Cfg><<<dim3((unsigned)nblk), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Split-KV partials: one block per (query block, head, batch x window),
+// fp32 O_s and LSE_s into the caller's workspace.
+template <class Cfg>
+int launch_fwd_split(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int Hq,
+                     int Hkv, int Nq, int Nk, float scale, int n_splits, int kv_chunk, DeviceState* st,
+                     cudaStream_t stream) {
+  static bool attr_set[kMaxDevices] = {};
+  int rc = set_smem_once(attn_fwd_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set);
+  if (rc != ATTN_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if ((rc = encode_qkv<Cfg>(&tq, &tk, &tv, q, k, v, B, Hq, Hkv, Nq, Nk)) != ATTN_OK) return rc;
+  FwdParams p;
+  if (!fill_params<Cfg>(&p, nullptr, nullptr, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr, nullptr, st))
+    return ATTN_ERR_UNSUPPORTED;
+  p.n_splits = n_splits;
+  p.kv_chunk = kv_chunk;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  const dim3 grid((unsigned)p.n_qblocks, (unsigned)Hq, (unsigned)(B * n_splits));
+  attn_fwd_kernel<Cfg><<<grid, Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <bool C> using CfgSplitD64 = FwdCfg<64, 128, 2, 3, 3, C, false, 3>;
+template <bool C> using CfgSplitD128 = FwdCfg<128, 128, 2, 2, 2, C, false, 2>;
+template <bool C> using CfgSplitD256 = FwdCfg<256, 64, 1, 2, 2, C, false, 0>;
+
+template <template <bool> class Cfg>
+int launch_split_causal(bool causal, const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                        int B, int Hq, int Hkv, int Nq, int Nk, float scale, int n_splits, int kv_chunk,
+                        DeviceState* st, cudaStream_t s) {
+  return causal ? launch_fwd_split<Cfg<true>>(q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, n_splits,
+                                              kv_chunk, st, s)
+                : launch_fwd_split<Cfg<false>>(q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, n_splits,
+                                               kv_chunk, st, s);
+}
+
+int launch_combine(const float* o_part, const float* lse_part, int S, int B, int Hq, int Nq, int d, void* o,
+                   float* lse, cudaStream_t s) {
+  const long long rows = (long long)B * Nq * Hq;
+  const long long blocks = (rows * 32 + 255) / 256;
+  if (blocks > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
+  auto* ob = reinterpret_cast<__nv_bfloat16*>(o);
+  switch (d) {
+    case 64: attn_combine_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(o_part, lse_part, S, B, Hq, Nq, ob, lse); break;
+    case 128: attn_combine_kernel<128><<<(unsigned)blocks, 256, 0, s>>>(o_part, lse_part, S, B, Hq, Nq, ob, lse); break;
+    default: attn_combine_kernel<256><<<(unsigned)blocks, 256, 0, s>>>(o_part, lse_part, S, B, Hq, Nq, ob, lse); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Split plan: windows of kv_chunk keys (a multiple of 128, so of every key
+// tile) and the number of non-empty windows.  n_splits <= 0 asks for enough
+// blocks to fill the GPU about twice, with windows of at least 512 keys.
+struct SplitPlan {
+  int n_splits, kv_chunk;
+};
+SplitPlan split_plan(int B, int Hq, int Nq, int Nk, int n_splits, int num_sms) {
+  if (n_splits <= 0) {
+    const long long blocks = (long long)B * Hq * ((Nq + 255) / 256);
+    long long want = (2ll * num_sms + blocks - 1) / (blocks > 0 ? blocks : 1);
+    const long long cap = Nk / 512 > 1 ? Nk / 512 : 1;
+    want = want < 1 ? 1 : (want > cap ? cap : want);
+    n_splits = (int)(want > 256 ? 256 : want);
+  }
+  if (n_splits > kMaxSplits) n_splits = kMaxSplits;
+  const long long per = (Nk + n_splits - 1) / n_splits;
+  const int chunk = (int)(((per + 127) / 128) * 128);
+  const int eff = chunk > 0 ? (int)((Nk + chunk - 1) / chunk) : 1;
+  return SplitPlan{eff < 1 ? 1 : eff, chunk > 0 ? chunk : 128};
+}
+long long splitkv_bytes(long long S, long long B, long long Hq, long long Nq, long long d) {
+  const long long o_bytes = ((S * B * Nq * Hq * d * 4) + 255) / 256 * 256;
+  return o_bytes + S * B * Hq * Nq * 4;
 }
 
 // Key ranges up to this length use the persistent kernel: their work items
@@ -373,6 +455,90 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float*
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
   return launch_sched<CfgFP8, CfgFP8>(causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, scale, descale_q, descale_k,
                                       descale_v, st, s);
+}
+
+long long attn_splitkv_workspace_bytes(int B, int Hq, int Nq, int Nk, int d, int n_splits) {
+  if (B < 0 || Hq < 0 || Nq < 0 || Nk < 0 || (d != 64 && d != 128 && d != 256)) return -1;
+  if (B == 0 || Hq == 0 || Nq == 0 || Nk == 0) return 0;
+  int num_sms = 148;
+  if (n_splits <= 0) {
+    int dev = 0;
+    DeviceState* st = nullptr;
+    if (device_state(&dev, &st) != ATTN_OK) return -1;
+    num_sms = st->num_sms;
+  }
+  const SplitPlan sp = split_plan(B, Hq, Nq, Nk, n_splits, num_sms);
+  if (sp.n_splits == 1) return 0;
+  return splitkv_bytes(sp.n_splits, B, Hq, Nq, d);
+}
+
+int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                     int Nq, int Nk, int d, int causal, float scale, int n_splits, void* workspace,
+                     long long workspace_bytes, void* stream) {
+  int rc = check_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, scale);
+  if (rc == -1) return ATTN_OK;
+  if (rc != ATTN_OK) return rc;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  int dev = 0;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
+  const SplitPlan sp = split_plan(B, Hq, Nq, Nk, n_splits, st->num_sms);
+  if (sp.n_splits == 1) return attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, ATTN_BF16, stream);
+  if ((long long)B * sp.n_splits > 65535) return ATTN_ERR_UNSUPPORTED;  // grid z
+  const long long need = splitkv_bytes(sp.n_splits, B, Hq, Nq, d);
+  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
+  float* o_part = static_cast<float*>(workspace);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             ((long long)sp.n_splits * B * Nq * Hq * d * 4 + 255) / 256 * 256);
+  const bool c = causal != 0;
+  switch (d) {
+    case 64:
+      rc = launch_split_causal<CfgSplitD64>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, sp.n_splits,
+                                            sp.kv_chunk, st, s);
+      break;
+    case 128:
+      rc = launch_split_causal<CfgSplitD128>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, sp.n_splits,
+                                             sp.kv_chunk, st, s);
+      break;
+    default:
+      rc = launch_split_causal<CfgSplitD256>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, sp.n_splits,
+                                             sp.kv_chunk, st, s);
+      break;
+  }
+  if (rc != ATTN_OK) return rc;
+  return launch_combine(o_part, lse_part, sp.n_splits, B, Hq, Nq, d, o, lse, s);
+}
+
+int attn_combine(const float* o_parts, const float* lse_parts, int n_splits, int B, int Hq, int Nq, int d, void* o,
+                 float* lse, void* stream) {
+  if (n_splits < 1 || B < 0 || Hq < 0 || Nq < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || Hq == 0 || Nq == 0) return ATTN_OK;
+  if (o_parts == nullptr || lse_parts == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(lse_parts) & 3u) != 0 ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0))
+    return ATTN_ERR_MISALIGNED;
+  int dev = 0;
+  DeviceState* st = nullptr;
+  int rc = device_state(&dev, &st);
+  if (rc != ATTN_OK) return rc;
+  return launch_combine(o_parts, lse_parts, n_splits, B, Hq, Nq, d, o, lse, static_cast<cudaStream_t>(stream));
+}
+
+int attn_kv_tile_count_window(int row0, int row1, int Nq, int Nk, int shift, int bn, int causal) {
+  if (row0 < 0 || row1 < row0 || Nq < 0 || Nk < 0 || shift < 0 || bn <= 0 || (causal != 0 && causal != 1)) return -1;
+  return kv_tile_count(row0, row1, Nq, Nk, bn, causal != 0, shift);
+}
+
+int attn_tile_kind_window(int row0, int row1, int kt, int Nq, int Nk, int shift, int bn, int causal) {
+  if (row0 < 0 || row1 < row0 || kt < 0 || Nq < 0 || Nk < 0 || shift < 0 || bn <= 0 ||
+      (causal != 0 && causal != 1))
+    return -1;
+  return tile_kind(row0, row1, kt, Nq, Nk, bn, causal != 0, shift);
 }
 
 long long attn_hadamard_quant_fp8_workspace_bytes(void) { return 256; }

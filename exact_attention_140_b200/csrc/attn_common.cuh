@@ -18,6 +18,15 @@ struct FwdParams {
   int n_items;      // B * Hq * n_qblocks work items
   int qb_major;     // 1: order items by query block (longest first) across heads; 0: head-major
   float sl2;        // scale * log2(e)
+  // split-KV (one-block-per-item kernel): the keys are cut into n_splits
+  // windows of kv_chunk keys (a multiple of the key tile); window s of batch b
+  // runs as grid z = b * n_splits + s and writes fp32 partials, O_s =
+  // o_part[s][b][row][h][:] (normalised by its own row sum) and LSE_s =
+  // lse_part[s][b][h][row].  n_splits = 1, kv_chunk = Nk, o_part = nullptr:
+  // no split, bf16 O written to o.
+  int n_splits, kv_chunk;
+  float* o_part;
+  float* lse_part;
   const float* dq;  // FP8 descales (device scalars), nullptr for bf16
   const float* dk;
   const float* dv;

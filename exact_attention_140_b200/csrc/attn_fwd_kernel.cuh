@@ -71,14 +71,19 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = p.n_qblocks - 1 - (int)blockIdx.x;  // longest causal blocks first
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.y;
+  const int b = (int)blockIdx.z / p.n_splits, split = (int)blockIdx.z % p.n_splits;
+  // key window of this block: [kv0, kv0 + nk), `shift` keys after it
+  const int kv0 = split * p.kv_chunk;
+  const int nk = p.Nk - kv0 < p.kv_chunk ? p.Nk - kv0 : p.kv_chunk;
+  const int shift = p.Nk - kv0 - nk;
   const int kh = h / p.group;
   const int q0 = qb * BM * NQT;
   int n_kv[NQT];
   int nmax = 0;
 #pragma unroll
   for (int t = 0; t < NQT; ++t) {
-    n_kv[t] = kv_tile_count(q0 + t * BM, q0 + (t + 1) * BM, p.Nq, p.Nk, BN, Cfg::CAUSAL);
+    n_kv[t] = kv_tile_count(q0 + t * BM, q0 + (t + 1) * BM, p.Nq, nk, BN, Cfg::CAUSAL, shift);
     nmax = n_kv[t] > nmax ? n_kv[t] : nmax;
   }
 
@@ -129,7 +134,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
     const uint32_t o_taddr = tmem + lane_off + (uint32_t)(Cfg::O_COL0 + t * D);
     float sl2 = p.sl2;
     if constexpr (Cfg::FP8) sl2 *= __ldg(p.dq) * __ldg(p.dk);
-    const long long vend = vis_end(row, p.Nq, p.Nk, Cfg::CAUSAL);
+    const long long vend = vis_end(row, p.Nq, nk, Cfg::CAUSAL, shift);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
@@ -139,7 +144,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       const uint32_t s_taddr = tmem + lane_off + (uint32_t)(si * BN);
-      const bool partial = tile_kind(row0, row0 + BM, j, p.Nq, p.Nk, BN, Cfg::CAUSAL) == kTilePartial;
+      const bool partial = tile_kind(row0, row0 + BM, j, p.Nq, nk, BN, Cfg::CAUSAL, shift) == kTilePartial;
       const int nvis = (int)(vend - (long long)j * BN);  // visible keys of this tile (masks partial tiles)
       // ---- one read of the whole score row (one TMEM load latency per tile)
       uint32_t sr[BN];
@@ -280,29 +285,50 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       const bool store = row < p.Nq;
       float inv = l > 0.f ? 1.f / l : 0.f;
       if constexpr (Cfg::FP8) inv *= __ldg(p.dv);
-      __nv_bfloat16* orow =
-          reinterpret_cast<__nv_bfloat16*>(p.o) + (((long long)b * p.Nq + row) * p.Hq + h) * (long long)D;
+      const float lse = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      if (p.o_part == nullptr) {
+        __nv_bfloat16* orow =
+            reinterpret_cast<__nv_bfloat16*>(p.o) + (((long long)b * p.Nq + row) * p.Hq + h) * (long long)D;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        if (nt > 0) {
-          ptx::tmem_ld32(o_taddr + 32 * c, r);
-          ptx::tmem_wait_ld_dep(r);
-        }
-        uint32_t w[16];
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          if (nt > 0) {
+            ptx::tmem_ld32(o_taddr + 32 * c, r);
+            ptx::tmem_wait_ld_dep(r);
+          }
+          uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = nt > 0 ? ptx::pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv)
-                        : 0u;
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+          for (int e = 0; e < 16; ++e)
+            w[e] = nt > 0 ? ptx::pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv)
+                          : 0u;
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
         }
-      }
-      if (store && p.lse != nullptr) {
-        const float lse = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
-        p.lse[((long long)b * p.Hq + h) * p.Nq + row] = lse;
+        if (store && p.lse != nullptr) p.lse[((long long)b * p.Hq + h) * p.Nq + row] = lse;
+      } else {
+        // split-KV partial of window `split`: fp32 O_s and LSE_s
+        const long long zs = (long long)split * p.B + b;
+        float* orow = p.o_part + ((zs * p.Nq + row) * p.Hq + h) * (long long)D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          if (nt > 0) {
+            ptx::tmem_ld32(o_taddr + 32 * c, r);
+            ptx::tmem_wait_ld_dep(r);
+          }
+          if (store) {
+            float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = nt > 0 ? make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                                            __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        if (store) p.lse_part[(zs * p.Hq + h) * p.Nq + row] = lse;
       }
     }
   } else if (warp == Cfg::TMA_WARP) {
@@ -336,7 +362,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
 #pragma unroll
           for (int c = 0; c < Cfg::NCH; ++c)
             ptx::tma_load_4d(sbase + Cfg::OFF_K + ks * Cfg::KV_BYTES + c * Cfg::CH_KV, &tmK, fb, c * Cfg::BOXE,
-                             kh, j * BN, b);
+                             kh, kv0 + j * BN, b);
           ++k_issued[ks];
         }
         const int vs = j % VST;
@@ -348,7 +374,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
 #pragma unroll
           for (int c = 0; c < Cfg::NCH; ++c)
             ptx::tma_load_4d(sbase + Cfg::OFF_V + vs * Cfg::KV_BYTES + c * Cfg::CH_KV, &tmV, fb, c * Cfg::BOXE,
-                             kh, j * BN, b);
+                             kh, kv0 + j * BN, b);
           ++v_issued[vs];
         }
       }

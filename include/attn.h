@@ -174,6 +174,59 @@ int attn_kv_tile_count(int row0, int row1, int Nq, int Nk, int bn, int causal);
 int attn_tile_kind(int row0, int row1, int kt, int Nq, int Nk, int bn, int causal);
 
 /*
+ * Split-KV forward (decode-shaped calls: few query rows, long key ranges).
+ * The same operation as attn_fwd (BF16, d in {64, 128, 256}, same layouts,
+ * causal rule and outputs), computed as n_splits partial attentions over
+ * contiguous key windows and merged by attn_combine's LSE-weighted sum; page
+ * "FlashAttention (SV)", section "Online-beräkning av Softmax" (the rescaling
+ * by exp(m_old - m_new) that lets partial results over key blocks merge);
+ * the pages name FlashDecoding for the decode setting but give no method, so
+ * the window split and the combine formula are this library's reading.
+ *   n_splits        requested number of key windows; <= 0 chooses one that
+ *                   fills the GPU about twice (windows of >= 512 keys).  The
+ *                   windows hold a multiple of 128 keys; fewer windows than
+ *                   requested may result.  One window runs attn_fwd itself.
+ *   workspace       DEVICE scratch, 16-byte aligned, of at least
+ *                   attn_splitkv_workspace_bytes(B, Hq, Nq, Nk, d, n_splits)
+ *                   bytes (0 when no split results: workspace may be NULL);
+ *                   owned by the caller, not retained after the call.
+ * Returns ATTN_ERR_INVALID_ARG for a missing or short workspace and
+ * ATTN_ERR_UNSUPPORTED when B * windows exceeds 65535; otherwise as attn_fwd.
+ * attn_splitkv_workspace_bytes returns -1 for invalid sizes (and, with
+ * n_splits <= 0, when no sm_100 device is current).
+ */
+long long attn_splitkv_workspace_bytes(int B, int Hq, int Nq, int Nk, int d, int n_splits);
+int attn_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                     int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                     int n_splits, void *workspace, long long workspace_bytes, void *stream);
+
+/*
+ * LSE-weighted merge of S partial results over disjoint key windows:
+ *   LSE = ln sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) * O_s
+ * (windows with LSE_s = -inf weigh nothing; a row whose every LSE_s is -inf
+ * gets O = 0, LSE = -inf).
+ *   o_parts    DEVICE fp32 [S, B, Nq, Hq, d]: O_s, each normalised by its own
+ *              row sum; 16-byte aligned
+ *   lse_parts  DEVICE fp32 [S, B, Hq, Nq]: LSE_s (natural log)
+ *   o          DEVICE bf16 [B, Nq, Hq, d], 16-byte aligned; lse DEVICE fp32
+ *              [B, Hq, Nq] or NULL
+ * Exported for callers that shard keys across devices and for the tests;
+ * attn_fwd_splitkv uses it on its own partials.
+ */
+int attn_combine(const float *o_parts, const float *lse_parts, int n_splits, int B, int Hq, int Nq,
+                 int d, void *o, float *lse, void *stream);
+
+/*
+ * The tile plan for a key window (split-KV): the window holds Nk keys and
+ * `shift` further keys follow it, so that in window-local indices query row i
+ * sees key j iff j < Nk and (!causal || j <= i + (Nk - Nq) + shift).
+ * shift = 0 is attn_kv_tile_count / attn_tile_kind.  Host-only; -1 on
+ * invalid arguments.
+ */
+int attn_kv_tile_count_window(int row0, int row1, int Nq, int Nk, int shift, int bn, int causal);
+int attn_tile_kind_window(int row0, int row1, int kt, int Nq, int Nk, int shift, int bn, int causal);
+
+/*
  * Which kernel attn_fwd / attn_fwd_fp8 launch for a key range of Nk keys:
  * 1 = the persistent kernel (one block per SM looping over the work items;
  * used for short key ranges, whose items are short), 0 = one block per work

@@ -68,3 +68,40 @@ def test_invalid_arguments():
     assert ea.attn_kv_tile_count(0, 5, 10, 10, 0, 0) == -1
     assert ea.attn_tile_kind(0, 5, -1, 10, 10, 64, 1) == -1
     assert ea.attn_tile_kind(0, 5, 0, 10, 10, 64, 3) == -1
+
+
+def check_window(Nq, nk, kv0, shift, bm, bn, causal):
+    """Keys [kv0, kv0 + nk) of a range of kv0 + nk + shift keys: the window's
+    plan against the window's columns of the full elementwise mask."""
+    mask = oracle.mask(Nq, kv0 + nk + shift, causal)[:, kv0:kv0 + nk]
+    n_q = (Nq + bm - 1) // bm + 1
+    for qt in range(n_q):
+        row0, row1 = qt * bm, (qt + 1) * bm
+        count, kinds = expected_plan(mask, row0, row1, bn)
+        got = ea.attn_kv_tile_count_window(row0, row1, Nq, nk, shift, bn, causal)
+        assert got == count, (Nq, nk, kv0, shift, bm, bn, causal, qt)
+        for kt, kd in enumerate(kinds):
+            assert ea.attn_tile_kind_window(row0, row1, kt, Nq, nk, shift, bn, causal) == kd, \
+                (Nq, nk, kv0, shift, bm, bn, causal, qt, kt)
+
+
+def test_key_windows():
+    rng = np.random.default_rng(141)
+    for _ in range(200):
+        Nq = int(rng.integers(1, 260))
+        nk = int(rng.integers(1, 300))
+        kv0, shift = int(rng.integers(0, 300)), int(rng.integers(0, 300))
+        bm, bn = int(rng.choice([64, 128])), int(rng.choice([64, 128]))
+        check_window(Nq, nk, kv0, shift, bm, bn, int(rng.integers(0, 2)))
+
+
+def test_window_without_shift_is_the_plain_plan():
+    for Nq, Nk in ((1, 1), (70, 300), (300, 70), (128, 256)):
+        for causal in (0, 1):
+            for kt in range(4):
+                assert ea.attn_tile_kind_window(0, 128, kt, Nq, Nk, 0, 64, causal) == \
+                    ea.attn_tile_kind(0, 128, kt, Nq, Nk, 64, causal)
+            assert ea.attn_kv_tile_count_window(0, 128, Nq, Nk, 0, 64, causal) == \
+                ea.attn_kv_tile_count(0, 128, Nq, Nk, 64, causal)
+    assert ea.attn_kv_tile_count_window(0, 5, 10, 10, -1, 64, 0) == -1
+    assert ea.attn_tile_kind_window(0, 5, 0, 10, 10, 0, 64, 2) == -1
