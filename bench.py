@@ -253,7 +253,7 @@ def run_ours(args, cfg, name):
                             desc.data_ptr() + 4, desc.data_ptr() + 8, stream)
         launches_per_step = 7  # 3 x (amax + quantise) + attention
     elif cfg.get("split"):
-        ws_bytes = ea.attn_splitkv_workspace_bytes(B, Hq, Nq, N, d, 0)
+        ws_bytes = ea.attn_splitkv_workspace_bytes(B, Hq, Hkv, Nq, N, d, 0)
         ws_split = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
 
         def step(qq, kk, vv):

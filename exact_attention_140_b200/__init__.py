@@ -70,7 +70,7 @@ _lib.attn_debug_unsatisfied_wait.argtypes = [_LL, _vp]
 _lib.attn_debug_unsatisfied_wait.restype = _I
 _lib.attn_debug_exp2.argtypes = [_vp, _vp, _LL, _I, _vp]
 _lib.attn_debug_exp2.restype = _I
-_lib.attn_splitkv_workspace_bytes.argtypes = [_I] * 6
+_lib.attn_splitkv_workspace_bytes.argtypes = [_I] * 7
 _lib.attn_splitkv_workspace_bytes.restype = _LL
 _lib.attn_fwd_splitkv.argtypes = [_vp] * 5 + [_I] * 7 + [_F, _I, _vp, _LL, _vp]
 _lib.attn_fwd_splitkv.restype = _I
@@ -122,8 +122,8 @@ def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype=ATTN_B
     return _check(rc, "attn_fwd", raise_on_error)
 
 
-def attn_splitkv_workspace_bytes(B, Hq, Nq, Nk, d, n_splits=0) -> int:
-    return int(_lib.attn_splitkv_workspace_bytes(B, Hq, Nq, Nk, d, n_splits))
+def attn_splitkv_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, n_splits=0) -> int:
+    return int(_lib.attn_splitkv_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, n_splits))
 
 
 def attn_fwd_splitkv(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, n_splits, workspace, workspace_bytes,

@@ -107,6 +107,24 @@ int encode_bnhd(CUtensorMap* m, const void* ptr, bool fp8, int B, int N, int H, 
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Q viewed as (d, g, Hkv, Nq, B) for head packing: a box of g heads x
+// rows / g query rows of one key/value head lands in shared memory as `rows`
+// packed 128-byte rows (row i * g + head-in-group), the layout of an unpacked
+// Q tile.
+int encode_q_packed(CUtensorMap* m, const void* ptr, int B, int Nq, int Hkv, int g, int d, int rows) {
+  const cuuint64_t es = 2;
+  const cuuint64_t Hq = (cuuint64_t)Hkv * g;
+  const cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)g, (cuuint64_t)Hkv, (cuuint64_t)Nq, (cuuint64_t)B};
+  const cuuint64_t strides[4] = {(cuuint64_t)d * es, (cuuint64_t)g * d * es, Hq * d * es,
+                                 (cuuint64_t)Nq * Hq * d * es};
+  const cuuint32_t box[5] = {(cuuint32_t)(128 / es), (cuuint32_t)g, 1u, (cuuint32_t)(rows / g), 1u};
+  const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 __global__ void empty_rows_kernel(__nv_bfloat16* o, float* lse, long long n_o, long long n_lse) {
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_o; i += (long long)gridDim.x * blockDim.x)
     o[i] = __float2bfloat16(0.f);
@@ -178,6 +196,7 @@ bool fill_params(FwdParams* p, void* o, float* lse, int B, int Hq, int Hkv, int 
   p->timeout_ns = timeout_ns();
   p->n_splits = 1;
   p->kv_chunk = Nk;
+  p->pack = 1;
   p->o_part = nullptr;
   p->lse_part = nullptr;
   return true;
@@ -245,13 +264,14 @@ int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, 
 // fp32 O_s and LSE_s into the caller's workspace.
 template <class Cfg>
 int launch_fwd_split(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int Hq,
-                     int Hkv, int Nq, int Nk, float scale, int n_splits, int kv_chunk, DeviceState* st,
+                     int Hkv, int Nq, int Nk, float scale, int n_splits, int kv_chunk, int pack, DeviceState* st,
                      cudaStream_t stream) {
   static bool attr_set[kMaxDevices] = {};
   int rc = set_smem_once(attn_fwd_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set);
   if (rc != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv;
   if ((rc = encode_qkv<Cfg>(&tq, &tk, &tv, q, k, v, B, Hq, Hkv, Nq, Nk)) != ATTN_OK) return rc;
+  if (pack > 1 && (rc = encode_q_packed(&tq, q, B, Nq, Hkv, pack, Cfg::D, Cfg::BM)) != ATTN_OK) return rc;
   FwdParams p;
   if (!fill_params<Cfg>(&p, nullptr, nullptr, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr, nullptr, st))
     return ATTN_ERR_UNSUPPORTED;
@@ -259,23 +279,33 @@ int launch_fwd_split(const void* q, const void* k, const void* v, float* o_part,
   p.kv_chunk = kv_chunk;
   p.o_part = o_part;
   p.lse_part = lse_part;
-  const dim3 grid((unsigned)p.n_qblocks, (unsigned)Hq, (unsigned)(B * n_splits));
+  p.pack = pack;
+  if (pack > 1) p.n_qblocks = (int)(((long long)Nq * pack + Cfg::BM * Cfg::NQT - 1) / (Cfg::BM * Cfg::NQT));
+  const dim3 grid((unsigned)p.n_qblocks, (unsigned)(pack > 1 ? Hkv : Hq), (unsigned)(B * n_splits));
   attn_fwd_kernel<Cfg><<<grid, Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <bool C> using CfgSplitD64 = FwdCfg<64, 128, 2, 3, 3, C, false, 3>;
-template <bool C> using CfgSplitD128 = FwdCfg<128, 128, 2, 2, 2, C, false, 2>;
-template <bool C> using CfgSplitD256 = FwdCfg<256, 64, 1, 2, 2, C, false, 0>;
+// the long-range configurations with head packing compiled in
+template <bool C> using CfgSplitD64 = FwdCfg<64, 128, 2, 3, 3, C, false, 3, 1, false, 1, true>;
+template <bool C> using CfgSplitD128 = FwdCfg<128, 128, 2, 2, 2, C, false, 2, 1, false, 1, true>;
+template <bool C> using CfgSplitD256 = FwdCfg<256, 64, 1, 2, 2, C, false, 0, 2, false, 1, true>;
 
 template <template <bool> class Cfg>
 int launch_split_causal(bool causal, const void* q, const void* k, const void* v, float* o_part, float* lse_part,
-                        int B, int Hq, int Hkv, int Nq, int Nk, float scale, int n_splits, int kv_chunk,
+                        int B, int Hq, int Hkv, int Nq, int Nk, float scale, int n_splits, int kv_chunk, int pack,
                         DeviceState* st, cudaStream_t s) {
   return causal ? launch_fwd_split<Cfg<true>>(q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, n_splits,
-                                              kv_chunk, st, s)
+                                              kv_chunk, pack, st, s)
                 : launch_fwd_split<Cfg<false>>(q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, n_splits,
-                                               kv_chunk, st, s);
+                                               kv_chunk, pack, st, s);
+}
+
+// Head packing for split-KV: the query heads of a key/value group share one
+// query tile when the group size divides the 128-row tile.
+int pack_factor(int Hq, int Hkv) {
+  const int g = Hq / Hkv;
+  return (g > 1 && 128 % g == 0) ? g : 1;
 }
 
 int launch_combine(const float* o_part, const float* lse_part, int S, int B, int Hq, int Nq, int d, void* o,
@@ -298,9 +328,10 @@ int launch_combine(const float* o_part, const float* lse_part, int S, int B, int
 struct SplitPlan {
   int n_splits, kv_chunk;
 };
-SplitPlan split_plan(int B, int Hq, int Nq, int Nk, int n_splits, int num_sms) {
+SplitPlan split_plan(int B, int Hq, int Hkv, int Nq, int Nk, int n_splits, int num_sms) {
   if (n_splits <= 0) {
-    const long long blocks = (long long)B * Hq * ((Nq + 255) / 256);
+    const int g = pack_factor(Hq, Hkv);
+    const long long blocks = (long long)B * (Hq / g) * (((long long)Nq * g + 255) / 256);
     long long want = (2ll * num_sms + blocks - 1) / (blocks > 0 ? blocks : 1);
     const long long cap = Nk / 512 > 1 ? Nk / 512 : 1;
     want = want < 1 ? 1 : (want > cap ? cap : want);
@@ -457,8 +488,9 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float*
                                       descale_v, st, s);
 }
 
-long long attn_splitkv_workspace_bytes(int B, int Hq, int Nq, int Nk, int d, int n_splits) {
-  if (B < 0 || Hq < 0 || Nq < 0 || Nk < 0 || (d != 64 && d != 128 && d != 256)) return -1;
+long long attn_splitkv_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int n_splits) {
+  if (B < 0 || Hq < 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq < 0 || Nk < 0 || (d != 64 && d != 128 && d != 256))
+    return -1;
   if (B == 0 || Hq == 0 || Nq == 0 || Nk == 0) return 0;
   int num_sms = 148;
   if (n_splits <= 0) {
@@ -467,7 +499,7 @@ long long attn_splitkv_workspace_bytes(int B, int Hq, int Nq, int Nk, int d, int
     if (device_state(&dev, &st) != ATTN_OK) return -1;
     num_sms = st->num_sms;
   }
-  const SplitPlan sp = split_plan(B, Hq, Nq, Nk, n_splits, num_sms);
+  const SplitPlan sp = split_plan(B, Hq, Hkv, Nq, Nk, n_splits, num_sms);
   if (sp.n_splits == 1) return 0;
   return splitkv_bytes(sp.n_splits, B, Hq, Nq, d);
 }
@@ -484,7 +516,7 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
-  const SplitPlan sp = split_plan(B, Hq, Nq, Nk, n_splits, st->num_sms);
+  const SplitPlan sp = split_plan(B, Hq, Hkv, Nq, Nk, n_splits, st->num_sms);
   if (sp.n_splits == 1) return attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, ATTN_BF16, stream);
   if ((long long)B * sp.n_splits > 65535) return ATTN_ERR_UNSUPPORTED;  // grid z
   const long long need = splitkv_bytes(sp.n_splits, B, Hq, Nq, d);
@@ -494,18 +526,19 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
   float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                              ((long long)sp.n_splits * B * Nq * Hq * d * 4 + 255) / 256 * 256);
   const bool c = causal != 0;
+  const int g = pack_factor(Hq, Hkv);
   switch (d) {
     case 64:
       rc = launch_split_causal<CfgSplitD64>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, sp.n_splits,
-                                            sp.kv_chunk, st, s);
+                                            sp.kv_chunk, g, st, s);
       break;
     case 128:
       rc = launch_split_causal<CfgSplitD128>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, sp.n_splits,
-                                             sp.kv_chunk, st, s);
+                                             sp.kv_chunk, g, st, s);
       break;
     default:
       rc = launch_split_causal<CfgSplitD256>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, sp.n_splits,
-                                             sp.kv_chunk, st, s);
+                                             sp.kv_chunk, g, st, s);
       break;
   }
   if (rc != ATTN_OK) return rc;

@@ -27,6 +27,12 @@ struct FwdParams {
   int n_splits, kv_chunk;
   float* o_part;
   float* lse_part;
+  // head packing (one-block-per-item kernel): pack = g > 1 stacks the g query
+  // heads of a key/value head in one query tile, packed row r = i * g + (h %
+  // g) (query row i); grid y is then the key/value head, n_qblocks counts
+  // tiles of packed rows, and Q is read through a 5-D map (d, g, Hkv, Nq, B).
+  // pack = 1: grid y is the query head.
+  int pack;
   const float* dq;  // FP8 descales (device scalars), nullptr for bf16
   const float* dk;
   const float* dv;
@@ -37,8 +43,11 @@ struct FwdParams {
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
 
 template <int D_, int BN_, int NQT_, int KST_, int VST_, bool CAUSAL_, bool FP8_, int EMU_ = 0,
-          int SB_ = (NQT_ == 1 ? 2 : 1), bool PSEP_ = false, int NS_ = 1>
+          int SB_ = (NQT_ == 1 ? 2 : 1), bool PSEP_ = false, int NS_ = 1, bool PACK_ = false>
 struct FwdCfg {
+  // PACK: the one-block-per-item kernel reads the head-packing factor from the
+  // launch parameters (split-KV); otherwise it is compiled out
+  static constexpr bool PACK = PACK_;
   static constexpr int D = D_, BN = BN_, NQT = NQT_, KST = KST_, VST = VST_;
   // NS: independent streams per block (persistent kernel): each has its own
   // softmax warpgroup(s), TMA and MMA warps, K/V rings, barriers and tensor

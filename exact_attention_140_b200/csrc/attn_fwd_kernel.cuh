@@ -71,19 +71,27 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = p.n_qblocks - 1 - (int)blockIdx.x;  // longest causal blocks first
-  const int h = blockIdx.y;
+  const int g = Cfg::PACK ? p.pack : 1;  // query heads stacked per tile row group
+  const int hy = blockIdx.y;         // query head, or key/value head when packed
   const int b = (int)blockIdx.z / p.n_splits, split = (int)blockIdx.z % p.n_splits;
   // key window of this block: [kv0, kv0 + nk), `shift` keys after it
   const int kv0 = split * p.kv_chunk;
   const int nk = p.Nk - kv0 < p.kv_chunk ? p.Nk - kv0 : p.kv_chunk;
   const int shift = p.Nk - kv0 - nk;
-  const int kh = h / p.group;
+  const int kh = g > 1 ? hy : hy / p.group;
   const int q0 = qb * BM * NQT;
   int n_kv[NQT];
   int nmax = 0;
+  // query rows [ia, ib) of tile t (packed rows r hold query row r / g)
+  auto tile_rows = [&](int t, int& ia, int& ib) {
+    ia = (q0 + t * BM) / g;
+    ib = (q0 + (t + 1) * BM + g - 1) / g;
+  };
 #pragma unroll
   for (int t = 0; t < NQT; ++t) {
-    n_kv[t] = kv_tile_count(q0 + t * BM, q0 + (t + 1) * BM, p.Nq, nk, BN, Cfg::CAUSAL, shift);
+    int ia, ib;
+    tile_rows(t, ia, ib);
+    n_kv[t] = kv_tile_count(ia, ib, p.Nq, nk, BN, Cfg::CAUSAL, shift);
     nmax = n_kv[t] > nmax ? n_kv[t] : nmax;
   }
 
@@ -127,8 +135,11 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
     // ------------------------------------------------------------ softmax
     if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_inc<Cfg::REG_SOFTMAX>();
     const int t = warp >> 2, wq = warp & 3;
-    const int row0 = q0 + t * BM;
-    const int row = row0 + wq * 32 + lane;
+    int ia, ib;
+    tile_rows(t, ia, ib);
+    const int prow = q0 + t * BM + wq * 32 + lane;  // this thread's (packed) tile row
+    const int row = prow / g;                         // its query row
+    const int h = g > 1 ? kh * g + (prow - row * g) : hy;
     const int nt = n_kv[t];
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t o_taddr = tmem + lane_off + (uint32_t)(Cfg::O_COL0 + t * D);
@@ -144,7 +155,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       const uint32_t s_taddr = tmem + lane_off + (uint32_t)(si * BN);
-      const bool partial = tile_kind(row0, row0 + BM, j, p.Nq, nk, BN, Cfg::CAUSAL, shift) == kTilePartial;
+      const bool partial = tile_kind(ia, ib, j, p.Nq, nk, BN, Cfg::CAUSAL, shift) == kTilePartial;
       const int nvis = (int)(vend - (long long)j * BN);  // visible keys of this tile (masks partial tiles)
       // ---- one read of the whole score row (one TMEM load latency per tile)
       uint32_t sr[BN];
@@ -348,9 +359,13 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         const uint32_t fb = bar(Cfg::B_QFULL + t);
         ptx::mbar_arrive_expect_tx(fb, Cfg::QT_BYTES);
 #pragma unroll
-        for (int c = 0; c < Cfg::NCH; ++c)
-          ptx::tma_load_4d(sbase + Cfg::OFF_Q + t * Cfg::QT_BYTES + c * Cfg::CH_Q, &tmQ, fb, c * Cfg::BOXE, h,
-                           q0 + t * BM, b);
+        for (int c = 0; c < Cfg::NCH; ++c) {
+          const uint32_t dst = sbase + Cfg::OFF_Q + t * Cfg::QT_BYTES + c * Cfg::CH_Q;
+          if (Cfg::PACK && g > 1)  // box: g heads x BM / g rows of kv head kh
+            ptx::tma_load_5d(dst, &tmQ, fb, c * Cfg::BOXE, 0, kh, (q0 + t * BM) / g, b);
+          else
+            ptx::tma_load_4d(dst, &tmQ, fb, c * Cfg::BOXE, hy, q0 + t * BM, b);
+        }
       }
       for (int j = 0; j < nmax; ++j) {
         const int ks = j % KST;

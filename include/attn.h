@@ -187,15 +187,19 @@ int attn_tile_kind(int row0, int row1, int kt, int Nq, int Nk, int bn, int causa
  *                   windows hold a multiple of 128 keys; fewer windows than
  *                   requested may result.  One window runs attn_fwd itself.
  *   workspace       DEVICE scratch, 16-byte aligned, of at least
- *                   attn_splitkv_workspace_bytes(B, Hq, Nq, Nk, d, n_splits)
+ *                   attn_splitkv_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, n_splits)
  *                   bytes (0 when no split results: workspace may be NULL);
  *                   owned by the caller, not retained after the call.
  * Returns ATTN_ERR_INVALID_ARG for a missing or short workspace and
  * ATTN_ERR_UNSUPPORTED when B * windows exceeds 65535; otherwise as attn_fwd.
+ * When the group size g = Hq / Hkv > 1 divides 128, the g query heads of a
+ * key/value head share query tiles (row i of head h at tile row i * g + h % g),
+ * so each key/value tile is read once per group and short query ranges fill
+ * the 128-row tiles.
  * attn_splitkv_workspace_bytes returns -1 for invalid sizes (and, with
  * n_splits <= 0, when no sm_100 device is current).
  */
-long long attn_splitkv_workspace_bytes(int B, int Hq, int Nq, int Nk, int d, int n_splits);
+long long attn_splitkv_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int n_splits);
 int attn_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
                      int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
                      int n_splits, void *workspace, long long workspace_bytes, void *stream);

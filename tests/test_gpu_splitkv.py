@@ -1,7 +1,9 @@
 """Split-KV on the GPU: the attention over key windows (fp32 partials) merged
 by the LSE-weighted combine, against the fp64 oracle of the unsplit
 definition (BF16 bar: max |dO| <= 1e-2, mean <= 1e-3, |dLSE| <= 1e-3); and the
-combine kernel alone against the oracle's merge."""
+combine kernel alone against the oracle's merge.  Grouped heads whose group
+size divides 128 run with their query heads stacked in one tile (head
+packing); the cases cover packed and unpacked groups."""
 import math
 
 import numpy as np
@@ -26,7 +28,7 @@ def run_splitkv(qb, kb, vb, causal, scale, n_splits):
     q, k, v = (to_dev_bf16(x) for x in (qb, kb, vb))
     o = T.full((B, Nq, Hq, d), float("nan"), dtype=T.bfloat16, device="cuda")
     lse = T.full((B, Hq, Nq), float("nan"), dtype=T.float32, device="cuda")
-    nbytes = ea.attn_splitkv_workspace_bytes(B, Hq, Nq, Nk, d, n_splits)
+    nbytes = ea.attn_splitkv_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, n_splits)
     assert nbytes >= 0
     ws = T.empty(max(nbytes, 16), dtype=T.uint8, device="cuda")
     ea.attn_fwd_splitkv(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, n_splits, ws, nbytes)
@@ -43,6 +45,10 @@ CASES = [  # d, B, Hq, Hkv, Nq, Nk, requested windows
     (64, 2, 4, 1, 16, 3000, 0),      # window count chosen by the library
     (128, 1, 2, 2, 128, 1024, 64),   # more windows asked than key tiles exist
     (128, 1, 2, 1, 200, 129, 2),     # causal: rows before the diagonal see nothing
+    (128, 1, 24, 8, 5, 3000, 4),     # group of 3 does not divide the tile: heads not packed
+    (64, 1, 16, 2, 9, 2500, 3),      # groups of 8 packed: 16 query rows per tile
+    (128, 1, 32, 1, 3, 1500, 2),     # MQA, group of 32: 96 packed rows in one tile
+    (256, 2, 8, 2, 40, 1200, 3),     # d = 256 with packing (one query tile per block)
 ]
 
 
@@ -114,7 +120,7 @@ def test_splitkv_argument_errors():
     q = T.zeros((1, 4, 2, 128), dtype=T.bfloat16, device="cuda")
     k = T.zeros((1, 4096, 2, 128), dtype=T.bfloat16, device="cuda")
     o = T.empty_like(q)
-    need = ea.attn_splitkv_workspace_bytes(1, 2, 4, 4096, 128, 4)
+    need = ea.attn_splitkv_workspace_bytes(1, 2, 2, 4, 4096, 128, 4)
     assert need > 0
     ws = T.empty(need, dtype=T.uint8, device="cuda")
     assert ea.attn_fwd_splitkv(q, k, k, o, None, 1, 2, 2, 4, 4096, 128, 0, 0.1, 4, ws, need - 1,
