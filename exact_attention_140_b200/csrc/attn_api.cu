@@ -286,9 +286,14 @@ int launch_fwd_split(const void* q, const void* k, const void* v, float* o_part,
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// the long-range configurations with head packing compiled in
+// the long-range configurations with head packing compiled in; when a key/
+// value group's (packed) query rows fit one 128-row tile, a block holds one
+// query tile with two score buffers instead (Q K_{j+1}^T under the softmax of
+// tile j), measured faster on decode shapes
 template <bool C> using CfgSplitD64 = FwdCfg<64, 128, 2, 3, 3, C, false, 3, 1, false, 1, true>;
 template <bool C> using CfgSplitD128 = FwdCfg<128, 128, 2, 2, 2, C, false, 2, 1, false, 1, true>;
+template <bool C> using CfgSplitD64One = FwdCfg<64, 128, 1, 3, 3, C, false, 3, 2, false, 1, true>;
+template <bool C> using CfgSplitD128One = FwdCfg<128, 128, 1, 2, 2, C, false, 2, 2, false, 1, true>;
 template <bool C> using CfgSplitD256 = FwdCfg<256, 64, 1, 2, 2, C, false, 0, 2, false, 1, true>;
 
 template <template <bool> class Cfg>
@@ -527,14 +532,19 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
                                              ((long long)sp.n_splits * B * Nq * Hq * d * 4 + 255) / 256 * 256);
   const bool c = causal != 0;
   const int g = pack_factor(Hq, Hkv);
+  const bool one_tile = (long long)Nq * g <= 128;
   switch (d) {
     case 64:
-      rc = launch_split_causal<CfgSplitD64>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, sp.n_splits,
-                                            sp.kv_chunk, g, st, s);
+      rc = one_tile ? launch_split_causal<CfgSplitD64One>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale,
+                                                          sp.n_splits, sp.kv_chunk, g, st, s)
+                    : launch_split_causal<CfgSplitD64>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale,
+                                                       sp.n_splits, sp.kv_chunk, g, st, s);
       break;
     case 128:
-      rc = launch_split_causal<CfgSplitD128>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, sp.n_splits,
-                                             sp.kv_chunk, g, st, s);
+      rc = one_tile ? launch_split_causal<CfgSplitD128One>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale,
+                                                           sp.n_splits, sp.kv_chunk, g, st, s)
+                    : launch_split_causal<CfgSplitD128>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale,
+                                                        sp.n_splits, sp.kv_chunk, g, st, s);
       break;
     default:
       rc = launch_split_causal<CfgSplitD256>(c, q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, scale, sp.n_splits,
