@@ -170,6 +170,27 @@ def oracle_sample(cfg, qb, kb, vb, target_s: float, n_rows: int | None = None, s
     return tf, desc, dt, n
 
 
+def rank_seed(rank: int) -> int:
+    """Input seed of a rank: every rank attends over its own batch (weak scaling)."""
+    return gen.BASE_SEED + 1000 * rank
+
+
+def max_over_ranks(values, device, world: int):
+    """Element-wise max of per-rank values (step counts, device times) over the
+    job; the only collective of a multi-GPU run, outside every timed region."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job rate: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank_step * steps * world / (max_ms * 1e-3)
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -225,7 +246,7 @@ def run_ours(args, cfg, name):
     scale = 1.0 / math.sqrt(d)
     fp8 = cfg["dtype"] == "fp8"
 
-    qb, kb, vb = make_inputs(cfg, seed=gen.BASE_SEED + 1000 * rank)
+    qb, kb, vb = make_inputs(cfg, seed=rank_seed(rank))
     host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (qb, kb, vb)]
     q, k, v = (h.to(dev) for h in host)
     o = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=dev)
@@ -277,10 +298,7 @@ def run_ours(args, cfg, name):
         w1.record(stream)
         torch.cuda.synchronize()
         per = w0.elapsed_time(w1) / 5 * 1e-3
-        t = torch.tensor([int(min(20000, max(20, 1.5 / per)))], device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        args.steps = int(t.item())
+        args.steps = int(max_over_ranks([int(min(20000, max(20, 1.5 / per)))], dev, world)[0])
     rc, word = ea.attn_get_last_device_error(stream)
     if rc != 0:
         raise RuntimeError(f"device error word {word:#x}")
@@ -334,18 +352,16 @@ def run_ours(args, cfg, name):
     torch.cuda.synchronize()
     e2e_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_st, e_en)))
 
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, world)
     if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.destroy_process_group()
-    total_ms, e2e_ms = float(t[0]), float(t[1])
     if rank != 0:
         return 0
 
     peaks = load_peaks()
     f = flops(cfg)
-    value = f * args.steps * world / (total_ms * 1e-3) / 1e12
-    e2e_value = f * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    value = job_throughput(f, args.steps, world, total_ms) / 1e12
+    e2e_value = job_throughput(f, e2e_steps, world, e2e_ms) / 1e12
     kern_avg_s = float(np.mean(kern_ms)) * 1e-3
     achieved = f / kern_avg_s / 1e12
     peak = peaks["bf16"] * (2.0 if fp8 else 1.0)
