@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   const int b = (int)(bi / Nq);
   const long long split_stride_lse = (long long)B * Hq * Nq;
   const long long lse_off = ((long long)b * Hq + h) * Nq + row;
+  // lane s holds LSE_s for the windows s, s + 32, ...; the row max first
   float m = -INFINITY;
   for (int s = lane; s < S; s += 32) m = fmaxf(m, __ldg(lse_part + s * split_stride_lse + lse_off));
 #pragma unroll
@@ -45,13 +46,32 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   if (m != -INFINITY) {
     const long long split_stride_o = rows * D;
     const float* src = o_part + warp * D + lane;
-    for (int s = 0; s < S; ++s) {
-      const float ls = __ldg(lse_part + s * split_stride_lse + lse_off);
-      if (ls == -INFINITY) continue;  // empty window (uniform across the warp)
-      const float w = expf(ls - m);
-      wsum += w;
+    // windows in groups of 32: each lane computes the weight of one window
+    // (0 for an empty window), then the group's weights are broadcast and its
+    // partial rows loaded 8 windows at a time, so the loads overlap
+    for (int s0 = 0; s0 < S; s0 += 32) {
+      const int sl = s0 + lane;
+      const float ls = sl < S ? __ldg(lse_part + sl * split_stride_lse + lse_off) : -INFINITY;
+      const float wl = ls == -INFINITY ? 0.f : expf(ls - m);
+      const int n = S - s0 < 32 ? S - s0 : 32;
+      for (int j0 = 0; j0 < n; j0 += 8) {
+        float w[8], x[8][PER];
 #pragma unroll
-      for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, __ldg(src + s * split_stride_o + 32 * e), acc[e]);
+        for (int u = 0; u < 8; ++u) {
+          w[u] = __shfl_sync(0xffffffffu, wl, (j0 + u) & 31);
+          const bool live = j0 + u < n && w[u] != 0.f;  // uniform across the warp
+#pragma unroll
+          for (int e = 0; e < PER; ++e)
+            x[u][e] = live ? __ldg(src + (long long)(s0 + j0 + u) * split_stride_o + 32 * e) : 0.f;
+          if (!live) w[u] = 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          wsum += w[u];
+#pragma unroll
+          for (int e = 0; e < PER; ++e) acc[e] = fmaf(w[u], x[u][e], acc[e]);
+        }
+      }
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
