@@ -39,6 +39,14 @@
 // softmax that skips most output rescalings).  The result is the same for any
 // TAU because the reference cancels in O = acc / l; TAU = 8 bounds P by 2^8.
 // Epilogue: O = O_t / l (bf16), LSE = ln2 * (m_ref + log2 l).
+//
+// Split-KV (launch parameters n_splits, kv_chunk, o_part, lse_part): a block
+// then covers one window of the keys (grid z = batch x window; the tile plan
+// is shifted so that the causal rule keeps absolute key indices) and writes
+// fp32 partials O_s = O_t / l and LSE_s for attn_combine.  With head packing
+// (PACK configurations, launch parameter pack = g) the g query heads of one
+// key/value head share the query tiles: query row i of head h sits at tile
+// row i * g + h % g, and grid y runs over key/value heads.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
