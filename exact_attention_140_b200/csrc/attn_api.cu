@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -212,15 +213,17 @@ int encode_qkv(CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv, const void* q,
   return ATTN_OK;
 }
 
-// Raises the kernel's dynamic shared memory limit once per device.
+// Raises the kernel's dynamic shared memory limit once per device (the flag
+// is atomic: concurrent first calls from several host threads both set the
+// same attribute, which is harmless).
 template <class Kernel>
-int set_smem_once(Kernel kernel, int bytes, bool (&done)[kMaxDevices]) {
+int set_smem_once(Kernel kernel, int bytes, std::atomic<bool> (&done)[kMaxDevices]) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
-  if (!done[dev]) {
+  if (!done[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_release);
   }
   return ATTN_OK;
 }
@@ -230,7 +233,7 @@ template <class Cfg>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
                int Nk, float scale, const float* dq, const float* dk, const float* dv, DeviceState* st,
                cudaStream_t stream) {
-  static bool attr_set[kMaxDevices] = {};
+  static std::atomic<bool> attr_set[kMaxDevices];
   int rc = set_smem_once(attn_fwd_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set);
   if (rc != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv;
@@ -247,7 +250,7 @@ template <class Cfg>
 int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                           int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
                           DeviceState* st, cudaStream_t stream) {
-  static bool attr_set[kMaxDevices] = {};
+  static std::atomic<bool> attr_set[kMaxDevices];
   int rc = set_smem_once(attn_fwd_persistent_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set);
   if (rc != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv;
@@ -266,7 +269,7 @@ template <class Cfg>
 int launch_fwd_split(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int Hq,
                      int Hkv, int Nq, int Nk, float scale, int n_splits, int kv_chunk, int pack, DeviceState* st,
                      cudaStream_t stream) {
-  static bool attr_set[kMaxDevices] = {};
+  static std::atomic<bool> attr_set[kMaxDevices];
   int rc = set_smem_once(attn_fwd_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set);
   if (rc != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv;
