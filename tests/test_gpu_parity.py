@@ -42,7 +42,7 @@ def test_several_tiles_ragged_tail(d, causal):
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("N", [1, 2, 17, 127, 129])
+@pytest.mark.parametrize("N", [1, 2, 17, 127, 129, 1000])
 @pytest.mark.parametrize("causal", [False, True])
 def test_odd_lengths(d, N, causal):
     full_check(1, 2, 2, N, N, d, causal)

@@ -55,9 +55,19 @@ def test_edge_shapes(bm, bn, causal):
             check(Nq, Nk, bm, bn, causal)
 
 
+@pytest.mark.parametrize("bn", [128, 64])
+@pytest.mark.parametrize("causal", [0, 1])
+def test_all_lengths_up_to_300(bn, causal):
+    """Exhaustive over Nq, Nk in [1, 300] for the kernels' tile shapes (128 query
+    rows; 128 keys, or 64 at d = 256)."""
+    for nq in range(1, 301):
+        for nk in range(1, 301):
+            check(nq, nk, 128, bn, causal)
+
+
 def test_random_shapes():
     rng = np.random.default_rng(140)
-    for _ in range(150):
+    for _ in range(1500):
         Nq, Nk = (int(x) for x in rng.integers(1, 301, size=2))
         bm, bn = int(rng.choice([64, 128])), int(rng.choice([64, 128]))
         check(Nq, Nk, bm, bn, int(rng.integers(0, 2)))
