@@ -95,3 +95,48 @@ def test_schedule_boundary():
     # persistent kernel for key ranges up to 1024, one block per item above
     assert ea.attn_fwd_schedule(-1) == -1
     assert [ea.attn_fwd_schedule(n) for n in (0, 1, 1024, 1025, 8192)] == [1, 1, 1, 0, 0]
+
+
+def test_splitkv_argument_errors_before_any_cuda_call():
+    def split(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=4, Hkv=2, Nq=8, Nk=4096, d=128, causal=0,
+                 scale=0.1, S=4, ws=FAKE, wsb=1 << 20)
+        a.update(kw)
+        return ea.attn_fwd_splitkv(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Nq"],
+                                   a["Nk"], a["d"], a["causal"], a["scale"], a["S"], a["ws"], a["wsb"], stream=0,
+                                   raise_on_error=False)
+    assert split(B=-1) == INVALID
+    assert split(Hq=3) == INVALID
+    assert split(causal=2) == INVALID
+    assert split(scale=float("nan")) == INVALID
+    assert split(o=0) == INVALID
+    assert split(q=FAKE + 8) == MISALIGNED
+    assert split(Nq=0) == OK  # nothing to compute
+
+
+def test_splitkv_workspace_sizes():
+    # windows of a multiple of 128 keys: 4096 keys in 4 windows of 1024
+    S, B, Hq, Nq, d = 4, 1, 4, 8, 128
+    o_bytes = (S * B * Nq * Hq * d * 4 + 255) // 256 * 256
+    assert ea.attn_splitkv_workspace_bytes(B, Hq, 2, Nq, 4096, d, S) == o_bytes + S * B * Hq * Nq * 4
+    # 300 keys asked for 8 windows: windows of 128 keys, 3 of them
+    assert ea.attn_splitkv_workspace_bytes(1, 2, 2, 4, 300, 64, 8) == (3 * 4 * 2 * 64 * 4 + 255) // 256 * 256 + 3 * 2 * 4 * 4
+    assert ea.attn_splitkv_workspace_bytes(1, 2, 2, 4, 100, 64, 8) == 0   # one window: no partials
+    assert ea.attn_splitkv_workspace_bytes(1, 2, 2, 4, 0, 64, 4) == 0     # no keys
+    assert ea.attn_splitkv_workspace_bytes(1, 3, 2, 4, 100, 64, 4) == -1  # Hq % Hkv != 0
+    assert ea.attn_splitkv_workspace_bytes(1, 2, 2, 4, 100, 96, 4) == -1  # head size
+
+
+def test_combine_argument_errors_before_any_cuda_call():
+    def comb(**kw):
+        a = dict(op=FAKE, lp=FAKE, S=3, B=1, Hq=2, Nq=5, d=128, o=FAKE, lse=FAKE)
+        a.update(kw)
+        return ea.attn_combine(a["op"], a["lp"], a["S"], a["B"], a["Hq"], a["Nq"], a["d"], a["o"], a["lse"],
+                               stream=0, raise_on_error=False)
+    assert comb(S=0) == INVALID
+    assert comb(B=-1) == INVALID
+    assert comb(d=96) == UNSUPPORTED
+    assert comb(op=0) == INVALID
+    assert comb(o=FAKE + 2) == MISALIGNED
+    assert comb(lse=FAKE + 2) == MISALIGNED
+    assert comb(Nq=0) == OK
