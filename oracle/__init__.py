@@ -61,6 +61,8 @@ def lib():
         L.oracle_attn_fwd_window.restype = _I
         L.oracle_combine.argtypes = [_dp, _dp, _I, _LL, _I, _dp, _dp]
         L.oracle_combine.restype = _I
+        L.oracle_gemm_add.argtypes = [_dp, _dp, ctypes.c_void_p, _dp, _LL, _LL, _LL]
+        L.oracle_gemm_add.restype = _I
         L.oracle_attn_bruteforce.argtypes = [_dp, _dp, _dp, _dp, _dp] + [_I] * 7 + [ctypes.c_double]
         L.oracle_attn_bruteforce.restype = _I
         L.oracle_mask.argtypes = [_I, _I, _I, _u8]
@@ -120,6 +122,21 @@ def attn_fwd_window(q, k, v, causal: bool, scale: float, k0: int, k1: int):
     if rc:
         raise ValueError(f"oracle_attn_fwd_window failed ({rc})")
     return o, lse
+
+
+def gemm_add(a, b, c=None):
+    """D = A B + C in fp64: a [M, K], b [K, N], c [M, N] or None."""
+    a, b = _f64(a), _f64(b)
+    M, K = a.shape
+    K2, N = b.shape
+    if K2 != K:
+        raise ValueError("inner sizes differ")
+    cc = None if c is None else _f64(c)
+    d = np.zeros((M, N))
+    cptr = None if cc is None else cc.ctypes.data_as(ctypes.c_void_p)
+    if lib().oracle_gemm_add(a, b, cptr, d, M, N, K):
+        raise ValueError("oracle_gemm_add failed")
+    return d
 
 
 def combine(o_parts, lse_parts):

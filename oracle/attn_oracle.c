@@ -53,6 +53,9 @@
  *                          list), ties to the even code, saturating to +-448.
  *   oracle_quant_e4m3_f32  per-tensor quantisation x * (448/amax) in fp32, then
  *                          E4M3 encode.
+ *   oracle_gemm_add        D = A B + C in fp64 (the small-K A@B+C workload page
+ *                          "FlashAttention-4震撼发布" names for Blackwell), rows
+ *                          of A [M, K], B [K, N], C and D [M, N], row-major.
  */
 #include <math.h>
 #include <stdint.h>
@@ -461,4 +464,23 @@ void oracle_e4m3_encode_array(const double *x, long long n, unsigned char *out)
 void oracle_e4m3_decode_array(const unsigned char *codes, long long n, double *out)
 {
     for (long long i = 0; i < n; ++i) out[i] = oracle_e4m3_decode(codes[i]);
+}
+
+/* D[m, n] = sum_k A[m, k] * B[k, n] + C[m, n] (C may be NULL: no addition).
+ * Plain fp64 sums in increasing k. */
+int oracle_gemm_add(const double *a, const double *b, const double *c, double *d,
+                    long long M, long long N, long long K)
+{
+    if (M < 0 || N < 0 || K < 0) return 1;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (long long m = 0; m < M; ++m) {
+        double *d_row = d + m * N;
+        for (long long n = 0; n < N; ++n) d_row[n] = c ? c[m * N + n] : 0.0;
+        for (long long k = 0; k < K; ++k) {
+            const double x = a[m * K + k];
+            const double *b_row = b + k * N;
+            for (long long n = 0; n < N; ++n) d_row[n] += x * b_row[n];
+        }
+    }
+    return 0;
 }
