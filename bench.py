@@ -37,6 +37,9 @@ sys.path.insert(0, ROOT)
 import attn_inputs as gen  # noqa: E402
 
 METRIC = "attn fwd TFLOP/s (4·B·H·N²·d, causal/2) and % of B200 dense BF16 peak"
+GEMM_METRIC = "A@B+C TFLOP/s (2·M·N·K)"
+# the small-K A@B+C workload (a separate line, not the attention metric)
+GEMM_WORKLOADS = {"gemm_add": dict(M=8192, N=8192, K=128)}
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -426,18 +429,148 @@ def traffic_bytes(name):
     return rec.get(name)
 
 
+def run_gemm(args, g, name):
+    """D = A B + C (bf16, fp32 accumulation): HBM-bound for small K, so the
+    roofline is bytes (A + B + C + D) over time.  --impl reference times the
+    fp64 oracle on a bounded sample of rows."""
+    M, N, K = g["M"], g["N"], g["K"]
+    ab, bb, cb = gen.normal_bf16(11, (M, K)), gen.normal_bf16(12, (K, N)), gen.normal_bf16(13, (M, N))
+    f = 2.0 * M * N * K
+
+    def oracle_rows(n_rows, seed):
+        import oracle
+        rows = np.sort(np.random.default_rng(seed).choice(M, size=n_rows, replace=False))
+        a64, b64, c64 = (gen.bf16_bits_to_f64(x) for x in (ab[rows], bb, cb[rows]))
+        t0 = time.perf_counter()
+        oracle.gemm_add(a64, b64, c64)
+        dt = time.perf_counter() - t0
+        return 2.0 * n_rows * N * K / dt / 1e12, f"{n_rows} of {M} rows of D (uniform sample), fp64; {dt:.1f} s"
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        steps = args.steps if args.steps > 0 else 3
+        vals = []
+        desc = ""
+        for i in range(args.warmup + steps):
+            tf, desc = oracle_rows(256, i)
+            if i >= args.warmup:
+                vals.append(tf)
+        v = float(statistics.median(vals))
+        print(json.dumps({
+            "impl": "reference", "metric": GEMM_METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": f / (v * 1e12) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{name}: M={M} N={N} K={K} bf16", "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_140_b200 as ea
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (ab, bb, cb)]
+    a, b, c = (h.to(dev) for h in host)
+    d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    d_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step(aa, bb_, cc):
+        ea.attn_gemm_add(aa, bb_, cc, d, M, N, K, stream)
+    for _ in range(max(3, args.warmup)):
+        step(a, b, c)
+    torch.cuda.synchronize()
+    if args.steps <= 0:
+        args.steps = 200
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            starts[i].record(stream)
+            step(a, b, c)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    rc, word = ea.attn_get_last_device_error(stream)
+    if rc != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+    step_ms = [x.elapsed_time(y) for x, y in zip(starts, ends)]
+    total_ms = float(sum(step_ms))
+    e2e_steps = max(3, min(args.steps, 20))
+    e_st = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e_en = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    da, db, dc = (torch.empty_like(x) for x in (a, b, c))
+    for i in range(e2e_steps):
+        e_st[i].record(stream)
+        da.copy_(host[0], non_blocking=True)
+        db.copy_(host[1], non_blocking=True)
+        dc.copy_(host[2], non_blocking=True)
+        step(da, db, dc)
+        d_host.copy_(d, non_blocking=True)
+        e_en[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = float(sum(x.elapsed_time(y) for x, y in zip(e_st, e_en)))
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, world)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peaks = load_peaks()
+    value = job_throughput(f, args.steps, world, total_ms) / 1e12
+    kern_s = total_ms / args.steps * 1e-3
+    alg_bytes = float(sum(x.numel() * x.element_size() for x in (a, b, c, d)))
+    line = {
+        "metric": GEMM_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{name}: M={M} N={N} K={K} bf16 (D = A B + C)",
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed between steps (256 MB write)"},
+        "roofline": {"bound": "hbm", "achieved": alg_bytes / kern_s / 1e9, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": alg_bytes / kern_s / 1e9 / peaks["hbm"], "traffic": traffic_bytes(name),
+                     "peak_source": f"{peaks['src']} hbm copy", "kernel": "gemm_add_kernel",
+                     "algorithmic_bytes": alg_bytes},
+        "e2e": {"value": job_throughput(f, e2e_steps, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in host)),
+                "d2h_bytes_per_step": int(d.numel() * d.element_size())},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        tf, desc = oracle_rows(256, 0)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=0, help="timed steps (0 = enough for about 1.5 s)")
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gpt2", choices=sorted(workloads()))
+    ap.add_argument("--workload", default="gpt2", choices=sorted(workloads()) + sorted(GEMM_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.workload in GEMM_WORKLOADS:
+        return run_gemm(args, GEMM_WORKLOADS[args.workload], args.workload)
     cfg = workloads()[args.workload]
     if args.impl == "reference":
         if args.steps <= 0:

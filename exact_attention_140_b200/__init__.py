@@ -19,8 +19,8 @@ __all__ = [
     "ATTN_BF16", "ATTN_FP8_E4M3", "AttnError", "attn_fwd", "attn_fwd_fp8", "attn_hadamard_quant_fp8",
     "attn_hadamard_quant_fp8_workspace_bytes", "attn_get_last_device_error", "attn_status_string",
     "attn_kv_tile_count", "attn_tile_kind", "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attention",
-    "attn_fwd_schedule",
-    "attn_hadamard_quant_fp8_noalloc", "lib_path", "EXPORTS",
+    "attn_fwd_schedule", "attn_hadamard_quant_fp8_noalloc", "attn_fwd_splitkv", "attn_splitkv_workspace_bytes",
+    "attn_combine", "attn_kv_tile_count_window", "attn_tile_kind_window", "attn_gemm_add", "lib_path", "EXPORTS",
 ]
 
 ATTN_BF16 = 0
@@ -37,7 +37,7 @@ EXPORTS = (
     "attn_get_last_device_error", "attn_status_string", "attn_kv_tile_count", "attn_tile_kind",
     "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attn_hadamard_quant_fp8_noalloc", "attn_fwd_schedule",
     "attn_fwd_splitkv", "attn_splitkv_workspace_bytes", "attn_combine", "attn_kv_tile_count_window",
-    "attn_tile_kind_window",
+    "attn_tile_kind_window", "attn_gemm_add",
 )
 
 if not os.path.exists(lib_path):
@@ -80,6 +80,8 @@ _lib.attn_kv_tile_count_window.argtypes = [_I] * 7
 _lib.attn_kv_tile_count_window.restype = _I
 _lib.attn_tile_kind_window.argtypes = [_I] * 8
 _lib.attn_tile_kind_window.restype = _I
+_lib.attn_gemm_add.argtypes = [_vp] * 4 + [_I] * 3 + [_vp]
+_lib.attn_gemm_add.restype = _I
 
 
 class AttnError(RuntimeError):
@@ -137,6 +139,11 @@ def attn_combine(o_parts, lse_parts, n_splits, B, Hq, Nq, d, o, lse, stream=None
     rc = _lib.attn_combine(_ptr(o_parts), _ptr(lse_parts), n_splits, B, Hq, Nq, d, _ptr(o), _ptr(lse),
                            _stream(stream))
     return _check(rc, "attn_combine", raise_on_error)
+
+
+def attn_gemm_add(a, b, c, d, M, N, K, stream=None, raise_on_error=True):
+    rc = _lib.attn_gemm_add(_ptr(a), _ptr(b), _ptr(c), _ptr(d), M, N, K, _stream(stream))
+    return _check(rc, "attn_gemm_add", raise_on_error)
 
 
 def attn_fwd_fp8(q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, descale_q, descale_k, descale_v,

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "attn.h"
@@ -15,6 +16,7 @@
 #include "attn_fwd_persistent_kernel.cuh"
 #include "combine.cuh"
 #include "fp8_prep.cuh"
+#include "gemm_add.cuh"
 #include "tiles.h"
 
 namespace attn {
@@ -121,6 +123,21 @@ int encode_q_packed(CUtensorMap* m, const void* ptr, int B, int Nq, int Hkv, int
   const cuuint32_t box[5] = {(cuuint32_t)(128 / es), (cuuint32_t)g, 1u, (cuuint32_t)(rows / g), 1u};
   const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
   const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// 2-D row-major bf16 matrix [rows, cols] as a 4-D map (cols, rows, 1, 1), box
+// (64 columns = 128 bytes, box_rows), 128-byte swizzle, zero fill out of range.
+int encode_rows(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows) {
+  const cuuint64_t es = 2;
+  const cuuint64_t dims[4] = {(cuuint64_t)cols, (cuuint64_t)rows, 1, 1};
+  const cuuint64_t row_bytes = (cuuint64_t)cols * es, all = (cuuint64_t)rows * row_bytes;
+  const cuuint64_t strides[3] = {row_bytes, all, all};
+  const cuuint32_t box[4] = {64u, (cuuint32_t)box_rows, 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
@@ -585,6 +602,43 @@ int attn_tile_kind_window(int row0, int row1, int kt, int Nq, int Nk, int shift,
       (causal != 0 && causal != 1))
     return -1;
   return tile_kind(row0, row1, kt, Nq, Nk, bn, causal != 0, shift);
+}
+
+int attn_gemm_add(const void* a, const void* b, const void* c, void* d, int M, int N, int K, void* stream) {
+  if (M < 0 || N < 0 || K < 0) return ATTN_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return ATTN_OK;
+  if (d == nullptr || (K > 0 && (a == nullptr || b == nullptr))) return ATTN_ERR_INVALID_ARG;
+  if (N % 8 != 0 || K % 8 != 0) return ATTN_ERR_UNSUPPORTED;  // 16-byte row strides for TMA and vector access
+  if ((K > 0 && (!aligned16(a) || !aligned16(b))) || (c != nullptr && !aligned16(c)) || !aligned16(d))
+    return ATTN_ERR_MISALIGNED;
+  int dev = 0;
+  DeviceState* st = nullptr;
+  int rc = device_state(&dev, &st);
+  if (rc != ATTN_OK) return rc;
+  static std::atomic<bool> attr_set[kMaxDevices];
+  if ((rc = set_smem_once(gemm_add_kernel, (int)GemmCfg::SMEM_BYTES, attr_set)) != ATTN_OK) return rc;
+  CUtensorMap ta, tb;
+  std::memset(&ta, 0, sizeof(ta));
+  std::memset(&tb, 0, sizeof(tb));
+  if (K > 0 && (encode_rows(&ta, a, M, K, GemmCfg::BM) != ATTN_OK || encode_rows(&tb, b, K, N, GemmCfg::BK) != ATTN_OK))
+    return ATTN_ERR_CUDA;
+  GemmParams p;
+  p.c = static_cast<const __nv_bfloat16*>(c);
+  p.d = static_cast<__nv_bfloat16*>(d);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.tiles_m = (M + GemmCfg::BM - 1) / GemmCfg::BM;
+  const long long tiles = (long long)p.tiles_m * ((N + GemmCfg::BN - 1) / GemmCfg::BN);
+  if (tiles > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
+  p.n_tiles = (int)tiles;
+  p.k_steps = (K + GemmCfg::BK - 1) / GemmCfg::BK;
+  p.err = st->err;
+  p.timeout_ns = timeout_ns();
+  const int nblk = p.n_tiles < st->num_sms ? p.n_tiles : st->num_sms;
+  gemm_add_kernel<<<dim3((unsigned)nblk), GemmCfg::NTHREADS, GemmCfg::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
+      ta, tb, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 long long attn_hadamard_quant_fp8_workspace_bytes(void) { return 256; }

@@ -1,0 +1,247 @@
+// gemm_add.cuh -- D = A B + C on tcgen05 for small reduction sizes K.
+//
+// Page "FlashAttention-4震撼发布" reports an A@B+C kernel for Blackwell that is
+// faster than the vendor library when K is small, by overlapping the epilogue
+// through two accumulation buffers; it gives no further detail, so this design
+// is ours.  With small K the work is the epilogue: reading C and writing D
+// (2 x 2 bytes per element) against 2K FLOPs per element, so the kernel is
+// HBM-bound and the tensor-core products must hide under the epilogue.
+//
+// Persistent grid (one block per SM, tiles of 128 x 256 in round-robin
+// order).  Warp roles:
+//   warps 0..7   epilogue, two warpgroups: warpgroup g takes columns
+//                [128 g, 128 g + 128) of the tile, warp w its TMEM lanes
+//                32 (w % 4) .. +31 (one tile row per thread); it reads the
+//                accumulator from TMEM, adds C and stores D (bf16);
+//   warp 8       TMA producer: A (K-major) and B (MN-major) tiles of BK = 64
+//                through a STAGES-deep shared-memory ring;
+//   warp 9       MMA issuer (converged warp, elected lane), also allocates
+//                tensor memory: tile i accumulates into TMEM columns
+//                [256 (i % 2), +256), so the products of tile i + 1 run while
+//                the epilogue drains tile i.
+// Layouts: A [M, K], B [K, N], C and D [M, N], row-major bf16; fp32
+// accumulation; D = bf16(A B + C) with round-to-nearest-even.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "attn_common.cuh"
+#include "ptx.cuh"
+
+namespace attn {
+
+struct GemmCfg {
+  static constexpr int BM = 128, BN = 256, BK = 64;
+  static constexpr int STAGES = 4;
+  static constexpr uint32_t A_BYTES = BM * 128;            // 128 rows of 64 bf16
+  static constexpr uint32_t B_CHUNK = BK * 128;            // 64 K-rows of 64 N-columns
+  static constexpr uint32_t B_BYTES = B_CHUNK * (BN / 64);
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int B_FULL = 0, B_EMPTY = STAGES, B_ACCF = 2 * STAGES, B_ACCE = 2 * STAGES + 2;
+  static constexpr int B_DRAIN = 2 * STAGES + 4, NBAR = 2 * STAGES + 5;
+  static constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr uint32_t OFF_SLOT = OFF_BAR + NBAR * 8;
+  static constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
+  static constexpr uint32_t SMEM_BYTES = OFF_ABORT + 4 + 1024;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per block");
+  static constexpr int EPI_WARPS = 8, TMA_WARP = 8, MMA_WARP = 9, NTHREADS = 384;
+  static constexpr int EPI_THREADS = 32 * EPI_WARPS;
+  static constexpr uint32_t IDESC = ptx::idesc<false>(BM, BN, true);  // B is MN-major
+};
+
+struct GemmParams {
+  const __nv_bfloat16* c;  // [M, N] or nullptr
+  __nv_bfloat16* d;        // [M, N]
+  int M, N, K;
+  int tiles_m, n_tiles, k_steps;
+  unsigned int* err;
+  unsigned long long timeout_ns;
+};
+
+__global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
+    gemm_add_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmParams p) {
+  using G = GemmCfg;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
+  const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw_u32);
+  auto bar = [&](int i) -> uint32_t { return sbase + G::OFF_BAR + 8u * (uint32_t)i; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sgen + G::OFF_ABORT);
+  const WaitCtx wc{abort_flag, p.err, p.timeout_ns};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto tile_at = [&](int k) -> int {
+    const long long t = (long long)blockIdx.x + (long long)k * gridDim.x;
+    return t < p.n_tiles ? (int)t : -1;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < G::STAGES; ++s) {
+      ptx::mbar_init(bar(G::B_FULL + s), 1);
+      ptx::mbar_init(bar(G::B_EMPTY + s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(bar(G::B_ACCF + a), 1);
+      ptx::mbar_init(bar(G::B_ACCE + a), G::EPI_THREADS);
+    }
+    ptx::mbar_init(bar(G::B_DRAIN), 1);
+    *abort_flag = 0u;
+    ptx::fence_mbar_init();
+  }
+  if (warp == G::TMA_WARP && lane == 0) {
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+  }
+  if (warp == G::MMA_WARP) {
+    ptx::tmem_alloc(sbase + G::OFF_SLOT, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sgen + G::OFF_SLOT);
+
+  if (warp < G::EPI_WARPS) {
+    // ------------------------------------------------------------ epilogue
+    const int wg = warp >> 2, wq = warp & 3;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int tile = tile_at(k);
+      if (tile < 0) break;
+      const int acc = k & 1;
+      ok = wait_bar<kRoleSoftmax>(bar(G::B_ACCF + acc), (uint32_t)((k >> 1) & 1), wc, kSiteODone);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const int m0 = (tile % p.tiles_m) * G::BM, n0 = (tile / p.tiles_m) * G::BN;
+      const int row = m0 + wq * 32 + lane;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        const int col0 = n0 + wg * 128 + 32 * c;
+        uint32_t r[32];
+        if (p.k_steps > 0) {
+          ptx::tmem_ld32(tmem + lane_off + (uint32_t)(acc * 256 + wg * 128 + 32 * c), r);
+          ptx::tmem_wait_ld_dep(r);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        }
+        if (row_ok) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int col = col0 + 8 * g;
+            if (col >= p.N) break;  // N is a multiple of 8: groups are whole
+            const long long off = (long long)row * p.N + col;
+            float cv[8];
+            if (p.c != nullptr) {
+              const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.c + off));
+              const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                cv[2 * e] = __uint_as_float(w4[e] << 16);
+                cv[2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) cv[e] = 0.f;
+            }
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = ptx::pack_bf16x2(__uint_as_float(r[8 * g + 2 * e]) + cv[2 * e],
+                                      __uint_as_float(r[8 * g + 2 * e + 1]) + cv[2 * e + 1]);
+            *reinterpret_cast<uint4*>(p.d + off) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      // this accumulator has been read out: tile k + 2 may overwrite it
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(G::B_ACCE + acc));
+    }
+  } else if (warp == G::TMA_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued[G::STAGES];
+#pragma unroll
+      for (int s = 0; s < G::STAGES; ++s) issued[s] = 0;
+      int it = 0;  // k-blocks issued into the ring, across tiles
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int tile = tile_at(k);
+        if (tile < 0) break;
+        const int m0 = (tile % p.tiles_m) * G::BM, n0 = (tile / p.tiles_m) * G::BN;
+        for (int kb = 0; kb < p.k_steps; ++kb, ++it) {
+          const int s = it % G::STAGES;
+          if (it >= G::STAGES &&
+              !wait_bar<kRoleProducer>(bar(G::B_EMPTY + s), (uint32_t)(((it / G::STAGES) - 1) & 1), wc,
+                                       kSiteKEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar(G::B_FULL + s);
+          const uint32_t st = sbase + (uint32_t)s * G::STAGE_BYTES;
+          ptx::mbar_arrive_expect_tx(fb, G::STAGE_BYTES);
+          ptx::tma_load_4d(st, &tmA, fb, kb * G::BK, m0, 0, 0);
+#pragma unroll
+          for (int c = 0; c < G::BN / 64; ++c)
+            ptx::tma_load_4d(st + G::A_BYTES + (uint32_t)c * G::B_CHUNK, &tmB, fb, n0 + 64 * c, kb * G::BK, 0, 0);
+          ++issued[s];
+        }
+      }
+      // every issued copy must land before the block may exit
+#pragma unroll
+      for (int s = 0; s < G::STAGES; ++s)
+        if (issued[s] > 0)
+          wait_bar<kRoleProducer>(bar(G::B_FULL + s), (uint32_t)((issued[s] - 1) & 1), wc, kSiteKFull);
+    }
+  } else if (warp == G::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    bool ok = true;
+    int it = 0;
+    for (int k = 0; ok; ++k) {
+      const int tile = tile_at(k);
+      if (tile < 0) break;
+      const int acc = k & 1;
+      if (k >= 2) {  // the epilogue of tile k - 2 must have read this accumulator
+        ok = wait_bar_warp<kRoleMma>(bar(G::B_ACCE + acc), (uint32_t)(((k >> 1) - 1) & 1), wc, kSiteODone);
+        if (!ok) break;
+        ptx::tc_fence_after();
+      }
+      const uint32_t d_t = tmem + (uint32_t)(acc * 256);
+      for (int kb = 0; kb < p.k_steps; ++kb, ++it) {
+        const int s = it % G::STAGES;
+        ok = wait_bar_warp<kRoleMma>(bar(G::B_FULL + s), (uint32_t)((it / G::STAGES) & 1), wc, kSiteKFull);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint32_t st = sbase + (uint32_t)s * G::STAGE_BYTES;
+        const uint64_t ad0 = ptx::sdesc_sw128(st, 16u, 1024u);
+        const uint64_t bd0 = ptx::sdesc_sw128(st + G::A_BYTES, G::B_CHUNK, 1024u);
+#pragma unroll
+        for (int kk = 0; kk < G::BK / 16; ++kk) {
+          const uint64_t ad = ad0 + (uint64_t)(((uint32_t)kk * 32u) >> 4);       // 32 bytes along a row
+          const uint64_t bd = bd0 + (uint64_t)(((uint32_t)kk * 16u * 128u) >> 4);  // 16 rows of 128 bytes
+          ptx::warp_mma_ss<false>(d_t, ad, bd, G::IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::warp_commit(bar(G::B_EMPTY + s));
+      }
+      if (!ok) break;
+      ptx::warp_commit(bar(G::B_ACCF + acc));
+    }
+    // all issued MMAs must finish before tensor memory is freed
+    ptx::warp_commit(bar(G::B_DRAIN));
+    wait_bar_warp<kRoleMma>(bar(G::B_DRAIN), 0u, wc, kSiteDrain);
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == G::MMA_WARP) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace attn

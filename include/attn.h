@@ -231,6 +231,20 @@ int attn_kv_tile_count_window(int row0, int row1, int Nq, int Nk, int shift, int
 int attn_tile_kind_window(int row0, int row1, int kt, int Nq, int Nk, int shift, int bn, int causal);
 
 /*
+ * attn_gemm_add -- D = A B + C for small reduction sizes K (page
+ * "FlashAttention-4震撼发布": an A@B+C kernel on Blackwell that overlaps its
+ * epilogue with the next products through two accumulation buffers; the page
+ * gives no sizes or method, so layouts and tiling are this library's).
+ *   a  [M, K] bf16, b [K, N] bf16, c [M, N] bf16 or NULL (no addition),
+ *   d  [M, N] bf16 output; all row-major DEVICE pointers, 16-byte aligned.
+ * Products accumulate in fp32; D = bf16(A B + C), round to nearest even.
+ * N and K must be multiples of 8 (ATTN_ERR_UNSUPPORTED otherwise); K = 0
+ * gives D = C (or 0).  Any M and N; any K, though the design targets small K
+ * (the kernel is then HBM-bound on reading C and writing D).
+ */
+int attn_gemm_add(const void *a, const void *b, const void *c, void *d, int M, int N, int K, void *stream);
+
+/*
  * Which kernel attn_fwd / attn_fwd_fp8 launch for a key range of Nk keys:
  * 1 = the persistent kernel (one block per SM looping over the work items;
  * used for short key ranges, whose items are short), 0 = one block per work

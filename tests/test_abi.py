@@ -140,3 +140,19 @@ def test_combine_argument_errors_before_any_cuda_call():
     assert comb(o=FAKE + 2) == MISALIGNED
     assert comb(lse=FAKE + 2) == MISALIGNED
     assert comb(Nq=0) == OK
+
+
+def test_gemm_add_argument_errors_before_any_cuda_call():
+    def g(**kw):
+        a = dict(a=FAKE, b=FAKE, c=FAKE, d=FAKE, M=128, N=256, K=64)
+        a.update(kw)
+        return ea.attn_gemm_add(a["a"], a["b"], a["c"], a["d"], a["M"], a["N"], a["K"], stream=0,
+                                raise_on_error=False)
+    assert g(M=-1) == INVALID
+    assert g(d=0) == INVALID
+    assert g(a=0) == INVALID
+    assert g(N=12) == UNSUPPORTED
+    assert g(K=60) == UNSUPPORTED
+    assert g(a=FAKE + 8) == MISALIGNED
+    assert g(c=FAKE + 2) == MISALIGNED
+    assert g(M=0) == OK and g(N=0) == OK
