@@ -111,14 +111,28 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
       const int tile = tile_at(k);
       if (tile < 0) break;
       const int acc = k & 1;
+      const int m0 = (tile % p.tiles_m) * G::BM, n0 = (tile / p.tiles_m) * G::BN;
+      const int row = m0 + wq * 32 + lane;
+      const bool row_ok = row < p.M;
+      const long long row_off = (long long)row * p.N;
+      // C does not depend on the products: this thread's 128 values of it are
+      // requested before the accumulator is waited for, so the loads overlap
+      // the wait and each other (N is a multiple of 8: 8-column groups are whole)
+      uint4 cr[4][4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int col = n0 + wg * 128 + 32 * c + 8 * g;
+          cr[c][g] = (p.c != nullptr && row_ok && col < p.N)
+                         ? __ldg(reinterpret_cast<const uint4*>(p.c + row_off + col))
+                         : make_uint4(0u, 0u, 0u, 0u);
+        }
       ok = wait_bar<kRoleSoftmax>(bar(G::B_ACCF + acc), (uint32_t)((k >> 1) & 1), wc, kSiteODone);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
-      const int m0 = (tile % p.tiles_m) * G::BM, n0 = (tile / p.tiles_m) * G::BN;
-      const int row = m0 + wq * 32 + lane;
-      const bool row_ok = row < p.M;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int col0 = n0 + wg * 128 + 32 * c;
         uint32_t r[32];
@@ -133,27 +147,15 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             const int col = col0 + 8 * g;
-            if (col >= p.N) break;  // N is a multiple of 8: groups are whole
-            const long long off = (long long)row * p.N + col;
-            float cv[8];
-            if (p.c != nullptr) {
-              const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.c + off));
-              const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+            if (col < p.N) {
+              const uint32_t w4[4] = {cr[c][g].x, cr[c][g].y, cr[c][g].z, cr[c][g].w};
+              uint32_t w[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                cv[2 * e] = __uint_as_float(w4[e] << 16);
-                cv[2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) cv[e] = 0.f;
+              for (int e = 0; e < 4; ++e)
+                w[e] = ptx::pack_bf16x2(__uint_as_float(r[8 * g + 2 * e]) + __uint_as_float(w4[e] << 16),
+                                        __uint_as_float(r[8 * g + 2 * e + 1]) + __uint_as_float(w4[e] & 0xFFFF0000u));
+              *reinterpret_cast<uint4*>(p.d + row_off + col) = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = ptx::pack_bf16x2(__uint_as_float(r[8 * g + 2 * e]) + cv[2 * e],
-                                      __uint_as_float(r[8 * g + 2 * e + 1]) + cv[2 * e + 1]);
-            *reinterpret_cast<uint4*>(p.d + off) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
