@@ -21,6 +21,7 @@ __all__ = [
     "attn_kv_tile_count", "attn_tile_kind", "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attention",
     "attn_fwd_schedule", "attn_hadamard_quant_fp8_noalloc", "attn_fwd_splitkv", "attn_splitkv_workspace_bytes",
     "attn_combine", "attn_kv_tile_count_window", "attn_tile_kind_window", "attn_gemm_add", "lib_path", "EXPORTS",
+    "attn_debug_map_cache_stats", "attn_fwd_part", "attn_shard_units", "attention_shard",
 ]
 
 ATTN_BF16 = 0
@@ -37,7 +38,7 @@ EXPORTS = (
     "attn_get_last_device_error", "attn_status_string", "attn_kv_tile_count", "attn_tile_kind",
     "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attn_hadamard_quant_fp8_noalloc", "attn_fwd_schedule",
     "attn_fwd_splitkv", "attn_splitkv_workspace_bytes", "attn_combine", "attn_kv_tile_count_window",
-    "attn_tile_kind_window", "attn_gemm_add",
+    "attn_tile_kind_window", "attn_gemm_add", "attn_debug_map_cache_stats", "attn_fwd_part", "attn_shard_units",
 )
 
 if not os.path.exists(lib_path):
@@ -48,6 +49,10 @@ _lib = ctypes.CDLL(lib_path)
 _vp, _I, _LL, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
 _lib.attn_fwd.argtypes = [_vp] * 5 + [_I] * 7 + [_F, _I, _vp]
 _lib.attn_fwd.restype = _I
+_lib.attn_fwd_part.argtypes = [_vp] * 5 + [_I] * 7 + [_F, _I] + [_I] * 4 + [_vp]
+_lib.attn_fwd_part.restype = _I
+_lib.attn_shard_units.argtypes = [_I] * 4 + [ctypes.POINTER(_I)]
+_lib.attn_shard_units.restype = _I
 _lib.attn_fwd_fp8.argtypes = [_vp] * 5 + [_I] * 7 + [_F, _vp, _vp, _vp, _vp]
 _lib.attn_fwd_fp8.restype = _I
 _lib.attn_hadamard_quant_fp8.argtypes = [_vp, _vp, _vp, _vp, _LL, _I, _vp, _vp]
@@ -82,6 +87,8 @@ _lib.attn_tile_kind_window.argtypes = [_I] * 8
 _lib.attn_tile_kind_window.restype = _I
 _lib.attn_gemm_add.argtypes = [_vp] * 4 + [_I] * 3 + [_vp]
 _lib.attn_gemm_add.restype = _I
+_lib.attn_debug_map_cache_stats.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)] * 2
+_lib.attn_debug_map_cache_stats.restype = _I
 
 
 class AttnError(RuntimeError):
@@ -122,6 +129,38 @@ def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype=ATTN_B
     rc = _lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, int(causal),
                        float(scale), int(dtype), _stream(stream))
     return _check(rc, "attn_fwd", raise_on_error)
+
+
+def attn_fwd_part(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype, b_begin, b_end, kvh_begin,
+                  kvh_end, stream=None, raise_on_error=True):
+    rc = _lib.attn_fwd_part(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, int(causal),
+                            float(scale), int(dtype), int(b_begin), int(b_end), int(kvh_begin), int(kvh_end),
+                            _stream(stream))
+    return _check(rc, "attn_fwd_part", raise_on_error)
+
+
+def attn_shard_units(B, Hkv, world, rank):
+    """Rank `rank`'s share of the B x Hkv (batch, key/value head) units as a list
+    of (b_begin, b_end, kvh_begin, kvh_end) rectangles."""
+    buf = (_I * 12)()
+    n = _lib.attn_shard_units(int(B), int(Hkv), int(world), int(rank), buf)
+    if n < 0:
+        raise AttnError(1, "attn_shard_units")
+    return [tuple(buf[4 * i:4 * i + 4]) for i in range(n)]
+
+
+def attention_shard(q, k, v, o, lse, rank, world, causal=False, scale=None, stream=None):
+    """This rank's share of attention over full bf16 tensors q [B,Nq,Hq,d],
+    k/v [B,Nk,Hkv,d] into o/lse (the other ranks' rows are not written);
+    returns the rectangles computed."""
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rects = attn_shard_units(B, Hkv, world, rank)
+    for (b0, b1, g0, g1) in rects:
+        attn_fwd_part(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, ATTN_BF16, b0, b1, g0, g1, stream)
+    return rects
 
 
 def attn_splitkv_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, n_splits=0) -> int:
@@ -201,6 +240,13 @@ def attn_fwd_schedule(Nk) -> int:
 def attn_debug_unsatisfied_wait(limit_ns: int, stream=None, raise_on_error=True):
     rc = _lib.attn_debug_unsatisfied_wait(int(limit_ns), _stream(stream))
     return _check(rc, "attn_debug_unsatisfied_wait", raise_on_error)
+
+
+def attn_debug_map_cache_stats():
+    """(hits, encodes) of the library's tensor-map cache."""
+    h, e = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+    _check(_lib.attn_debug_map_cache_stats(ctypes.byref(h), ctypes.byref(e)), "attn_debug_map_cache_stats", True)
+    return h.value, e.value
 
 
 def attn_debug_exp2(x, y, n, mode, stream=None, raise_on_error=True):

@@ -40,7 +40,11 @@ struct DeviceState {
   bool init = false;
   int status = ATTN_OK;
   unsigned int* err = nullptr;
+  unsigned int* noalloc_scratch = nullptr;  // device address of g_noalloc_scratch
+  const float* unit_descale = nullptr;      // device address of g_unit_descale
   int num_sms = 0;
+  CUcontext ctx = nullptr;  // context the addresses above belong to
+  unsigned gen = 0;         // bumped whenever the state is (re)built
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -48,7 +52,9 @@ std::mutex g_mu;
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
 EncodeTiledFn g_encode = nullptr;
+CtxGetCurrentFn g_ctx_current = nullptr;
 
 unsigned long long timeout_ns() {
   static unsigned long long v = [] {
@@ -60,54 +66,146 @@ unsigned long long timeout_ns() {
   return v;
 }
 
-// Per-device setup: checks for an sm_100 device and finds the error word.
+template <class Fn>
+bool driver_entry(const char* name, Fn* out) {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess ||
+      fn == nullptr)
+    return false;
+  *out = reinterpret_cast<Fn>(fn);
+  return true;
+}
+
+// Per-device setup: checks for an sm_100 device and finds the device
+// addresses of the library's own device variables.  The state belongs to the
+// device's current context: when that context changes (a cudaDeviceReset
+// destroys it) the state is rebuilt, so no address of an old context is used.
+// Only a verdict that cannot change (not an sm_100 device) is cached; a failed
+// CUDA call is retried on the next entry.
 int device_state(int* dev_out, DeviceState** st_out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceState& st = g_dev[dev];
-  if (!st.init) {
-    st.init = true;
-    int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-      st.status = ATTN_ERR_CUDA;
-    } else if (major != 10 || minor != 0) {
-      st.status = ATTN_ERR_UNSUPPORTED;  // built for sm_100a only
-    } else if (cudaGetSymbolAddress(reinterpret_cast<void**>(&st.err), g_err_word) != cudaSuccess) {
-      st.status = ATTN_ERR_CUDA;
-    }
-    if (st.status == ATTN_OK && g_encode == nullptr) {
-      void* fn = nullptr;
-      cudaDriverEntryPointQueryResult q;
-      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-          q != cudaDriverEntryPointSuccess || fn == nullptr)
-        st.status = ATTN_ERR_CUDA;
-      else
-        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-    }
-  }
   *dev_out = dev;
   *st_out = &st;
-  return st.status;
+  if (st.init && st.status == ATTN_OK) {
+    CUcontext cur = nullptr;
+    if (g_ctx_current(&cur) == CUDA_SUCCESS && cur == st.ctx) return ATTN_OK;
+    st.init = false;  // new context: look everything up again
+  }
+  if (st.init) return st.status;
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (major != 10 || minor != 0) {  // built for sm_100a only
+    st.init = true;
+    st.status = ATTN_ERR_UNSUPPORTED;
+    return st.status;
+  }
+  if ((g_encode == nullptr && !driver_entry("cuTensorMapEncodeTiled", &g_encode)) ||
+      (g_ctx_current == nullptr && !driver_entry("cuCtxGetCurrent", &g_ctx_current)))
+    return ATTN_ERR_CUDA;
+  unsigned int *err = nullptr, *scratch = nullptr;
+  float* one = nullptr;
+  // (these calls also create the device's context if it does not exist yet)
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_word) != cudaSuccess ||
+      cudaGetSymbolAddress(reinterpret_cast<void**>(&scratch), g_noalloc_scratch) != cudaSuccess ||
+      cudaGetSymbolAddress(reinterpret_cast<void**>(&one), g_unit_descale) != cudaSuccess || err == nullptr ||
+      scratch == nullptr || one == nullptr)
+    return ATTN_ERR_CUDA;
+  CUcontext cur = nullptr;
+  if (g_ctx_current(&cur) != CUDA_SUCCESS || cur == nullptr) return ATTN_ERR_CUDA;
+  st.err = err;
+  st.noalloc_scratch = scratch;
+  st.unit_descale = one;
+  st.num_sms = sms;
+  st.ctx = cur;
+  ++st.gen;
+  st.status = ATTN_OK;
+  st.init = true;
+  return ATTN_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// 4-D tiled map over a [B, N, H, d] tensor: dims (d, H, N, B), box
-// (128 bytes of d, 1 head, rows, 1), 128-byte swizzle, zero fill out of range.
+// Cache of encoded tensor maps.  A map is a pure function of the encoding's
+// arguments (base address, data type, dims, strides, box; the other fields
+// are the same for every map here), so a hit returns exactly what a fresh
+// encoding would; calls that reuse the same tensors skip the host-side
+// encoding.  kMapSets sets of kMapWays entries (round-robin replacement within
+// a set, so the few maps of one call never evict each other), guarded by a
+// mutex.
+struct MapKey {
+  uint64_t ptr;
+  uint32_t dtype, rank;
+  cuuint64_t dims[5], strides[4];
+  cuuint32_t box[5];
+};
+constexpr int kMapSets = 64, kMapWays = 4;
+struct MapEntry {
+  bool valid = false;
+  MapKey key;
+  CUtensorMap map;
+};
+struct MapSet {
+  MapEntry way[kMapWays];
+  int next = 0;
+};
+MapSet g_maps[kMapSets];
+std::mutex g_maps_mu;
+std::atomic<unsigned long long> g_map_hits{0}, g_map_encodes{0};
+
+int encode_cached(CUtensorMap* m, CUtensorMapDataType dt, uint32_t rank, const void* ptr, const cuuint64_t* dims,
+                  const cuuint64_t* strides, const cuuint32_t* box) {
+  MapKey key;
+  std::memset(&key, 0, sizeof(key));  // padding bytes take part in the comparison
+  key.ptr = reinterpret_cast<uint64_t>(ptr);
+  key.dtype = (uint32_t)dt;
+  key.rank = rank;
+  for (uint32_t i = 0; i < rank; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+    if (i + 1 < rank) key.strides[i] = strides[i];
+  }
+  uint64_t h = 1469598103934665603ull;  // FNV-1a over the key bytes
+  const unsigned char* kb = reinterpret_cast<const unsigned char*>(&key);
+  for (size_t i = 0; i < sizeof(key); ++i) h = (h ^ kb[i]) * 1099511628211ull;
+  MapSet& set = g_maps[h % kMapSets];
+  {
+    std::lock_guard<std::mutex> lk(g_maps_mu);
+    for (int w = 0; w < kMapWays; ++w)
+      if (set.way[w].valid && std::memcmp(&set.way[w].key, &key, sizeof(key)) == 0) {
+        *m = set.way[w].map;
+        g_map_hits.fetch_add(1, std::memory_order_relaxed);
+        return ATTN_OK;
+      }
+  }
+  const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+  const CUresult r = g_encode(m, dt, rank, const_cast<void*>(ptr), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return ATTN_ERR_CUDA;
+  g_map_encodes.fetch_add(1, std::memory_order_relaxed);
+  std::lock_guard<std::mutex> lk(g_maps_mu);
+  MapEntry& e = set.way[set.next];
+  set.next = (set.next + 1) % kMapWays;
+  e.valid = true;
+  std::memcpy(&e.key, &key, sizeof(key));
+  e.map = *m;
+  return ATTN_OK;
+}
+
 int encode_bnhd(CUtensorMap* m, const void* ptr, bool fp8, int B, int N, int H, int d, int rows) {
   const cuuint64_t es = fp8 ? 1 : 2;
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
   const cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)H * d * es, (cuuint64_t)N * H * d * es};
   const cuuint32_t box[4] = {(cuuint32_t)(128 / es), 1u, (cuuint32_t)rows, 1u};
-  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-  const CUresult r = g_encode(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
-                              const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+  return encode_cached(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims,
+                       strides, box);
 }
 
 // Q viewed as (d, g, Hkv, Nq, B) for head packing: a box of g heads x
@@ -121,11 +219,7 @@ int encode_q_packed(CUtensorMap* m, const void* ptr, int B, int Nq, int Hkv, int
   const cuuint64_t strides[4] = {(cuuint64_t)d * es, (cuuint64_t)g * d * es, Hq * d * es,
                                  (cuuint64_t)Nq * Hq * d * es};
   const cuuint32_t box[5] = {(cuuint32_t)(128 / es), (cuuint32_t)g, 1u, (cuuint32_t)(rows / g), 1u};
-  const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
-  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box,
-                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+  return encode_cached(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, ptr, dims, strides, box);
 }
 
 // 2-D row-major bf16 matrix [rows, cols] as a 4-D map (cols, rows, 1, 1), box
@@ -136,20 +230,23 @@ int encode_rows(CUtensorMap* m, const void* ptr, int rows, int cols, int box_row
   const cuuint64_t row_bytes = (cuuint64_t)cols * es, all = (cuuint64_t)rows * row_bytes;
   const cuuint64_t strides[3] = {row_bytes, all, all};
   const cuuint32_t box[4] = {64u, (cuuint32_t)box_rows, 1u, 1u};
-  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
-                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+  return encode_cached(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides, box);
 }
 
-__global__ void empty_rows_kernel(__nv_bfloat16* o, float* lse, long long n_o, long long n_lse) {
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_o; i += (long long)gridDim.x * blockDim.x)
-    o[i] = __float2bfloat16(0.f);
-  if (lse != nullptr)
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_lse;
-         i += (long long)gridDim.x * blockDim.x)
-      lse[i] = -INFINITY;
+// Rows that see no key (Nk == 0): O = 0 and LSE = -inf for batches
+// [b0, b0 + nb) and query heads [h0, h0 + nh) of the [B, Nq, Hq, d] output.
+__global__ void empty_rows_kernel(__nv_bfloat16* o, float* lse, int Nq, int Hq, int d, int b0, int nb, int h0,
+                                  int nh) {
+  const long long rows = (long long)nb * Nq * nh;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < rows * d; i += stride) {
+    const long long r = i / d;
+    const int c = (int)(i - r * d), h = h0 + (int)(r % nh);
+    const long long bi = r / nh;
+    const int b = b0 + (int)(bi / Nq), row = (int)(bi % Nq);
+    o[(((long long)b * Nq + row) * Hq + h) * d + c] = __float2bfloat16(0.f);
+    if (lse != nullptr && c == 0) lse[((long long)b * Hq + h) * Nq + row] = -INFINITY;
+  }
 }
 
 __global__ void unsatisfied_wait_kernel(unsigned int* err, unsigned long long limit_ns) {
@@ -183,11 +280,17 @@ __global__ void exp2_probe_kernel(const float* x, float* y, long long n, int mod
   if (i + 1 < n) y[i + 1] = yb;
 }
 
+// The part of a call's problem one launch computes: batches [b0, b0 + nb) and
+// query heads [h0, h0 + nh) (whole key/value groups).
+struct Part {
+  int b0, nb, h0, nh;
+};
+
 // Fills the parameters both kernels share; false when the work items do not
 // fit the kernels' int indexing.
 template <class Cfg>
 bool fill_params(FwdParams* p, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
-                 const float* dq, const float* dk, const float* dv, DeviceState* st) {
+                 const float* dq, const float* dk, const float* dv, DeviceState* st, const Part& part) {
   p->o = o;
   p->lse = lse;
   p->B = B;
@@ -196,15 +299,19 @@ bool fill_params(FwdParams* p, void* o, float* lse, int B, int Hq, int Hkv, int 
   p->Nq = Nq;
   p->Nk = Nk;
   p->group = Hq / Hkv;
+  p->b0 = part.b0;
+  p->nb = part.nb;
+  p->h0 = part.h0;
+  p->nh = part.nh;
   p->n_qblocks = (Nq + Cfg::BM * Cfg::NQT - 1) / (Cfg::BM * Cfg::NQT);
-  const long long items = (long long)B * Hq * p->n_qblocks;
+  const long long items = (long long)part.nb * part.nh * p->n_qblocks;
   if (items > 0x7FFFFFFFll) return false;
   p->n_items = (int)items;
   // causal blocks differ in length: the persistent kernel orders them
   // longest-first across heads when all of K and V fits comfortably in L2;
   // otherwise it keeps a head's query blocks together so that they share its
   // K/V tiles through L2
-  const long long kv_bytes = 2ll * B * Nk * Hkv * Cfg::D * Cfg::ELEM;
+  const long long kv_bytes = 2ll * part.nb * Nk * (part.nh / p->group) * Cfg::D * Cfg::ELEM;
   p->qb_major = (Cfg::CAUSAL && kv_bytes <= (48ll << 20)) ? 1 : 0;
   p->sl2 = scale * 1.4426950408889634f;
   p->dq = dq;
@@ -230,17 +337,18 @@ int encode_qkv(CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv, const void* q,
   return ATTN_OK;
 }
 
-// Raises the kernel's dynamic shared memory limit once per device (the flag
-// is atomic: concurrent first calls from several host threads both set the
-// same attribute, which is harmless).
+// Raises the kernel's dynamic shared memory limit once per device state (the
+// attribute belongs to the context, so a rebuilt state sets it again;
+// concurrent first calls from several host threads both set the same
+// attribute, which is harmless).
 template <class Kernel>
-int set_smem_once(Kernel kernel, int bytes, std::atomic<bool> (&done)[kMaxDevices]) {
+int set_smem_once(Kernel kernel, int bytes, std::atomic<unsigned> (&done)[kMaxDevices], const DeviceState* st) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
-  if (!done[dev].load(std::memory_order_acquire)) {
+  if (done[dev].load(std::memory_order_acquire) != st->gen) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    done[dev].store(true, std::memory_order_release);
+    done[dev].store(st->gen, std::memory_order_release);
   }
   return ATTN_OK;
 }
@@ -249,15 +357,15 @@ int set_smem_once(Kernel kernel, int bytes, std::atomic<bool> (&done)[kMaxDevice
 template <class Cfg>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
                int Nk, float scale, const float* dq, const float* dk, const float* dv, DeviceState* st,
-               cudaStream_t stream) {
-  static std::atomic<bool> attr_set[kMaxDevices];
-  int rc = set_smem_once(attn_fwd_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set);
+               cudaStream_t stream, const Part& part) {
+  static std::atomic<unsigned> attr_set[kMaxDevices];
+  int rc = set_smem_once(attn_fwd_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set, st);
   if (rc != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv;
   if ((rc = encode_qkv<Cfg>(&tq, &tk, &tv, q, k, v, B, Hq, Hkv, Nq, Nk)) != ATTN_OK) return rc;
   FwdParams p;
-  if (!fill_params<Cfg>(&p, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st)) return ATTN_ERR_UNSUPPORTED;
-  const dim3 grid((unsigned)p.n_qblocks, (unsigned)Hq, (unsigned)B);
+  if (!fill_params<Cfg>(&p, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, part)) return ATTN_ERR_UNSUPPORTED;
+  const dim3 grid((unsigned)p.n_qblocks, (unsigned)part.nh, (unsigned)part.nb);
   attn_fwd_kernel<Cfg><<<grid, Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -266,14 +374,14 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 template <class Cfg>
 int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                           int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
-                          DeviceState* st, cudaStream_t stream) {
-  static std::atomic<bool> attr_set[kMaxDevices];
-  int rc = set_smem_once(attn_fwd_persistent_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set);
+                          DeviceState* st, cudaStream_t stream, const Part& part) {
+  static std::atomic<unsigned> attr_set[kMaxDevices];
+  int rc = set_smem_once(attn_fwd_persistent_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set, st);
   if (rc != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv;
   if ((rc = encode_qkv<Cfg>(&tq, &tk, &tv, q, k, v, B, Hq, Hkv, Nq, Nk)) != ATTN_OK) return rc;
   FwdParams p;
-  if (!fill_params<Cfg>(&p, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st)) return ATTN_ERR_UNSUPPORTED;
+  if (!fill_params<Cfg>(&p, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, part)) return ATTN_ERR_UNSUPPORTED;
   const int nstreams = (p.n_items + Cfg::NS - 1) / Cfg::NS;  // blocks that find work
   const int nblk = nstreams < st->num_sms ? nstreams : st->num_sms;
   attn_fwd_persistent_kernel<Cfg><<<dim3((unsigned)nblk), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
@@ -286,14 +394,15 @@ template <class Cfg>
 int launch_fwd_split(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int Hq,
                      int Hkv, int Nq, int Nk, float scale, int n_splits, int kv_chunk, int pack, DeviceState* st,
                      cudaStream_t stream) {
-  static std::atomic<bool> attr_set[kMaxDevices];
-  int rc = set_smem_once(attn_fwd_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set);
+  static std::atomic<unsigned> attr_set[kMaxDevices];
+  int rc = set_smem_once(attn_fwd_kernel<Cfg>, (int)Cfg::SMEM_BYTES, attr_set, st);
   if (rc != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv;
   if ((rc = encode_qkv<Cfg>(&tq, &tk, &tv, q, k, v, B, Hq, Hkv, Nq, Nk)) != ATTN_OK) return rc;
   if (pack > 1 && (rc = encode_q_packed(&tq, q, B, Nq, Hkv, pack, Cfg::D, Cfg::BM)) != ATTN_OK) return rc;
   FwdParams p;
-  if (!fill_params<Cfg>(&p, nullptr, nullptr, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr, nullptr, st))
+  if (!fill_params<Cfg>(&p, nullptr, nullptr, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr, nullptr, st,
+                        Part{0, B, 0, Hq}))
     return ATTN_ERR_UNSUPPORTED;
   p.n_splits = n_splits;
   p.kv_chunk = kv_chunk;
@@ -395,13 +504,15 @@ template <bool C> using CfgFP8 = FwdCfg<128, 128, 2, 3, 3, C, true, 3>;
 template <template <bool> class Long, template <bool> class Short>
 int launch_sched(bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                  int Hkv, int Nq, int Nk, float scale, const float* dq, const float* dk, const float* dv,
-                 DeviceState* st, cudaStream_t s) {
+                 DeviceState* st, cudaStream_t s, const Part& pt) {
   const bool persist = Nk <= kPersistentMaxNk;
   if (causal)
-    return persist ? launch_fwd_persistent<Short<true>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
-                   : launch_fwd<Long<true>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
-  return persist ? launch_fwd_persistent<Short<false>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s)
-                 : launch_fwd<Long<false>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s);
+    return persist
+               ? launch_fwd_persistent<Short<true>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s, pt)
+               : launch_fwd<Long<true>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s, pt);
+  return persist
+             ? launch_fwd_persistent<Short<false>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s, pt)
+             : launch_fwd<Long<false>>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s, pt);
 }
 
 int check_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
@@ -418,10 +529,118 @@ int check_common(const void* q, const void* k, const void* v, void* o, float* ls
   return ATTN_OK;
 }
 
-int fill_empty(void* o, float* lse, int B, int Hq, int Nq, int d, cudaStream_t s) {
-  const long long n_o = (long long)B * Nq * Hq * d, n_lse = (long long)B * Hq * Nq;
-  empty_rows_kernel<<<256, 256, 0, s>>>(reinterpret_cast<__nv_bfloat16*>(o), lse, n_o, n_lse);
+__global__ void set_float_kernel(float* p, float v) { *p = v; }
+
+// FP8 preparation of one tensor [rows, 128] (both entry points): clear the
+// amax word, the amax pass, the quantising pass.  `amax` is one word of
+// device scratch (the caller's workspace or the library's static array).
+template <bool ROT>
+int launch_prep_passes(const CUtensorMap& tx, const CUtensorMap& tx8, const PrepParams& p, int grid, DeviceState* st,
+                       cudaStream_t s) {
+  static std::atomic<unsigned> attr_a[kMaxDevices], attr_q[kMaxDevices];
+  int rc;
+  if ((rc = set_smem_once(fp8_prep_kernel<ROT, false>, (int)PrepCfg<false>::SMEM_BYTES, attr_a, st)) != ATTN_OK ||
+      (rc = set_smem_once(fp8_prep_kernel<ROT, true>, (int)PrepCfg<true>::SMEM_BYTES, attr_q, st)) != ATTN_OK)
+    return rc;
+  fp8_prep_kernel<ROT, false><<<grid, kPrepRows, PrepCfg<false>::SMEM_BYTES, s>>>(tx, tx8, p);
+  fp8_prep_kernel<ROT, true><<<grid, kPrepRows, PrepCfg<true>::SMEM_BYTES, s>>>(tx, tx8, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int launch_prep(const void* x, void* x8, float* descale, unsigned int* amax, long long rows, const float* signs,
+                DeviceState* st, cudaStream_t s) {
+  if (rows == 0) {  // amax of nothing is 0: descale 1, as for an all-zero tensor
+    set_float_kernel<<<1, 1, 0, s>>>(descale, 1.0f);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  if (rows > 0x7FFFFFFFll - kPrepRows) return ATTN_ERR_UNSUPPORTED;  // tile coordinates are int
+  CUtensorMap tx, tx8;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)kPrepD, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kPrepD * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)kPrepRows};
+    if (encode_cached(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dims, strides, box) != ATTN_OK)
+      return ATTN_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)kPrepD, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kPrepD};
+    const cuuint32_t box[2] = {(cuuint32_t)kPrepD, (cuuint32_t)kPrepRows};
+    if (encode_cached(&tx8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, x8, dims, strides, box) != ATTN_OK)
+      return ATTN_ERR_CUDA;
+  }
+  PrepParams p;
+  p.rows = rows;
+  p.n_tiles = (int)((rows + kPrepRows - 1) / kPrepRows);
+  p.signs = signs;
+  p.amax_bits = amax;
+  p.descale = descale;
+  p.err = st->err;
+  p.timeout_ns = timeout_ns();
+  const int grid = p.n_tiles < 2 * st->num_sms ? p.n_tiles : 2 * st->num_sms;  // two blocks per SM
+  if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), s) != cudaSuccess) return ATTN_ERR_CUDA;
+  return signs != nullptr ? launch_prep_passes<true>(tx, tx8, p, grid, st, s)
+                          : launch_prep_passes<false>(tx, tx8, p, grid, st, s);
+}
+
+int fill_empty(void* o, float* lse, int B, int Hq, int Nq, int d, const Part& pt, cudaStream_t s) {
+  empty_rows_kernel<<<256, 256, 0, s>>>(reinterpret_cast<__nv_bfloat16*>(o), lse, Nq, Hq, d, pt.b0, pt.nb, pt.h0,
+                                        pt.nh);
+  (void)B;
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// The forward over one part of the problem, after the argument checks: the
+// kernel configuration for (d, dtype), short key ranges on the persistent
+// kernel.  fp8: E4M3 inputs with device descales dq, dk, dv.
+int fwd_checked(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                int Nk, int d, bool causal, float scale, bool fp8, const float* dq, const float* dk,
+                const float* dv, const Part& pt, DeviceState* st, cudaStream_t s) {
+  if (pt.nb == 0 || pt.nh == 0) return ATTN_OK;
+  if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, pt, s);
+  if (fp8) return launch_sched<CfgFP8, CfgFP8>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, s, pt);
+  switch (d) {
+    case 64:
+      return launch_sched<CfgD64, CfgD64Short>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr,
+                                               nullptr, st, s, pt);
+    case 128:
+      return launch_sched<CfgD128, CfgD128Short>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr,
+                                                 nullptr, st, s, pt);
+    default:
+      return launch_sched<CfgD256, CfgD256>(causal, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr,
+                                            nullptr, st, s, pt);
+  }
+}
+
+// Contiguous share of the B x Hkv (batch, key/value head) units, batch-major,
+// as up to three rectangles [b0, b1) x [g0, g1).
+int shard_rects(int B, int Hkv, int world, int rank, int* r) {
+  const long long U = (long long)B * Hkv;
+  const long long u0 = U * rank / world, u1 = U * (rank + 1) / world;
+  if (u0 >= u1) return 0;
+  const int bs = (int)(u0 / Hkv), gs = (int)(u0 % Hkv);
+  const int be = (int)((u1 - 1) / Hkv), ge = (int)((u1 - 1) % Hkv) + 1;
+  int n = 0;
+  auto put = [&](int b0, int b1, int g0, int g1) {
+    r[4 * n] = b0;
+    r[4 * n + 1] = b1;
+    r[4 * n + 2] = g0;
+    r[4 * n + 3] = g1;
+    ++n;
+  };
+  if (bs == be) {
+    put(bs, bs + 1, gs, ge);
+    return n;
+  }
+  int full0 = bs, full1 = be + 1;
+  if (gs > 0) {
+    put(bs, bs + 1, gs, Hkv);
+    full0 = bs + 1;
+  }
+  if (ge < Hkv) full1 = be;
+  if (full0 < full1) put(full0, full1, 0, Hkv);
+  if (ge < Hkv) put(be, be + 1, 0, ge);
+  return n;
 }
 
 }  // namespace
@@ -457,43 +676,34 @@ int attn_tile_kind(int row0, int row1, int kt, int Nq, int Nk, int bn, int causa
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk,
              int d, int causal, float scale, int dtype, void* stream) {
+  return attn_fwd_part(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype, 0, B, 0, Hkv, stream);
+}
+
+int attn_fwd_part(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                  int Nk, int d, int causal, float scale, int dtype, int b_begin, int b_end, int kvh_begin,
+                  int kvh_end, void* stream) {
   if (dtype != ATTN_BF16 && dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
-  if (dtype == ATTN_FP8_E4M3) {
-    // e4m3 inputs with unit scales: attn_fwd_fp8 with descales read from a
-    // device constant 1.0 (argument checks come before any CUDA call)
-    int rc = check_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, scale);
-    if (rc == -1) return ATTN_OK;
-    if (rc != ATTN_OK) return rc;
-    if (d != 128) return ATTN_ERR_UNSUPPORTED;
-    int dev = 0;
-    DeviceState* st = nullptr;
-    if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
-    void* one = nullptr;
-    if (cudaGetSymbolAddress(&one, g_unit_descale) != cudaSuccess) return ATTN_ERR_CUDA;
-    const float* u = static_cast<const float*>(one);
-    return attn_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, u, u, u, stream);
-  }
   int rc = check_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, scale);
   if (rc == -1) return ATTN_OK;
   if (rc != ATTN_OK) return rc;
-  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if (b_begin < 0 || b_end < b_begin || b_end > B || kvh_begin < 0 || kvh_end < kvh_begin || kvh_end > Hkv)
+    return ATTN_ERR_INVALID_ARG;
+  const bool fp8 = dtype == ATTN_FP8_E4M3;
+  if (fp8 ? d != 128 : (d != 64 && d != 128 && d != 256)) return ATTN_ERR_UNSUPPORTED;
   int dev = 0;
   DeviceState* st = nullptr;
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
-  const bool c = causal != 0;
-  switch (d) {
-    case 64:
-      return launch_sched<CfgD64, CfgD64Short>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr, nullptr,
-                                               st, s);
-    case 128:
-      return launch_sched<CfgD128, CfgD128Short>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr,
-                                                 nullptr, st, s);
-    default:
-      return launch_sched<CfgD256, CfgD256>(c, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, nullptr, nullptr, nullptr,
-                                            st, s);
-  }
+  const int g = Hq / Hkv;
+  const Part pt{b_begin, b_end - b_begin, kvh_begin * g, (kvh_end - kvh_begin) * g};
+  // e4m3 inputs with unit scales read the library's device constant 1.0
+  const float* u = fp8 ? st->unit_descale : nullptr;
+  return fwd_checked(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal != 0, scale, fp8, u, u, u, pt, st,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int attn_shard_units(int B, int Hkv, int world, int rank, int* rects) {
+  if (B < 0 || Hkv < 0 || world < 1 || rank < 0 || rank >= world || rects == nullptr) return -1;
+  return shard_rects(B, Hkv, world, rank, rects);
 }
 
 int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
@@ -507,10 +717,8 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float*
   int dev = 0;
   DeviceState* st = nullptr;
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
-  return launch_sched<CfgFP8, CfgFP8>(causal != 0, q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, scale, descale_q, descale_k,
-                                      descale_v, st, s);
+  return fwd_checked(q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, d, causal != 0, scale, true, descale_q, descale_k,
+                     descale_v, Part{0, B, 0, Hq}, st, static_cast<cudaStream_t>(stream));
 }
 
 long long attn_splitkv_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int n_splits) {
@@ -540,7 +748,7 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
   DeviceState* st = nullptr;
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, s);
+  if (Nk == 0) return fill_empty(o, lse, B, Hq, Nq, d, Part{0, B, 0, Hq}, s);
   const SplitPlan sp = split_plan(B, Hq, Hkv, Nq, Nk, n_splits, st->num_sms);
   if (sp.n_splits == 1) return attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, ATTN_BF16, stream);
   if ((long long)B * sp.n_splits > 65535) return ATTN_ERR_UNSUPPORTED;  // grid z
@@ -611,12 +819,17 @@ int attn_gemm_add(const void* a, const void* b, const void* c, void* d, int M, i
   if (N % 8 != 0 || K % 8 != 0) return ATTN_ERR_UNSUPPORTED;  // 16-byte row strides for TMA and vector access
   if ((K > 0 && (!aligned16(a) || !aligned16(b))) || (c != nullptr && !aligned16(c)) || !aligned16(d))
     return ATTN_ERR_MISALIGNED;
+  if (c != nullptr && c != d) {  // C may be D itself, but not partly overlap it
+    const uintptr_t cb = reinterpret_cast<uintptr_t>(c), db = reinterpret_cast<uintptr_t>(d);
+    const uintptr_t bytes = (uintptr_t)M * (uintptr_t)N * 2u;
+    if (cb < db + bytes && db < cb + bytes) return ATTN_ERR_INVALID_ARG;
+  }
   int dev = 0;
   DeviceState* st = nullptr;
   int rc = device_state(&dev, &st);
   if (rc != ATTN_OK) return rc;
-  static std::atomic<bool> attr_set[kMaxDevices];
-  if ((rc = set_smem_once(gemm_add_kernel, (int)GemmCfg::SMEM_BYTES, attr_set)) != ATTN_OK) return rc;
+  static std::atomic<unsigned> attr_set[kMaxDevices];
+  if ((rc = set_smem_once(gemm_add_kernel, (int)GemmCfg::SMEM_BYTES, attr_set, st)) != ATTN_OK) return rc;
   CUtensorMap ta, tb;
   std::memset(&ta, 0, sizeof(ta));
   std::memset(&tb, 0, sizeof(tb));
@@ -654,16 +867,8 @@ int attn_hadamard_quant_fp8(const void* x, void* x8, float* descale, void* works
   int dev = 0, rc;
   DeviceState* st = nullptr;
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  unsigned int* amax = static_cast<unsigned int*>(workspace);
-  if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), s) != cudaSuccess) return ATTN_ERR_CUDA;
-  const long long blocks_needed = (rows + kPrepWarps - 1) / kPrepWarps;
-  const long long cap = (long long)st->num_sms * 16;
-  const unsigned grid = (unsigned)(blocks_needed < 1 ? 1 : (blocks_needed < cap ? blocks_needed : cap));
-  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  fp8_amax_kernel<<<grid, 32 * kPrepWarps, 0, s>>>(xb, rows, signs, amax);
-  fp8_quant_kernel<<<grid, 32 * kPrepWarps, 0, s>>>(xb, rows, signs, amax, static_cast<uint8_t*>(x8), descale);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return launch_prep(x, x8, descale, static_cast<unsigned int*>(workspace), rows, signs, st,
+                     static_cast<cudaStream_t>(stream));
 }
 
 int attn_hadamard_quant_fp8_noalloc(const void* x, void* x8, float* descale, long long rows, int d,
@@ -679,29 +884,12 @@ int attn_hadamard_quant_fp8_noalloc(const void* x, void* x8, float* descale, lon
   int dev = 0, rc;
   DeviceState* st = nullptr;
   if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
-  // Host code cannot use g_noalloc_scratch's name as a device address: look the
-  // address up once per device, with that device current (the first call on a
-  // device does this).
-  static unsigned int* scratch[kMaxDevices] = {};
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (scratch[dev] == nullptr) {
-      void* ptr = nullptr;
-      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return ATTN_ERR_CUDA;
-      scratch[dev] = static_cast<unsigned int*>(ptr);
-    }
-  }
-  unsigned int* amax = scratch[dev];
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // The array keeps the previous call's maximum: clear it first.
-  if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), s) != cudaSuccess) return ATTN_ERR_CUDA;
-  const long long blocks_needed = (rows + kPrepWarps - 1) / kPrepWarps;
-  const long long cap = (long long)st->num_sms * 16;
-  const unsigned grid = (unsigned)(blocks_needed < 1 ? 1 : (blocks_needed < cap ? blocks_needed : cap));
-  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  fp8_amax_kernel<<<grid, 32 * kPrepWarps, 0, s>>>(xb, rows, signs, amax);
-  fp8_quant_kernel<<<grid, 32 * kPrepWarps, 0, s>>>(xb, rows, signs, amax, static_cast<uint8_t*>(x8), descale);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  // Host code cannot use g_noalloc_scratch's name as a device address: its
+  // address was looked up by device_state, once per device (and context), with
+  // that device current (the first call on a device does this).
+  // launch_prep clears the word it uses (the array keeps the previous call's
+  // maximum) before the amax pass.
+  return launch_prep(x, x8, descale, st->noalloc_scratch, rows, signs, st, static_cast<cudaStream_t>(stream));
 }
 
 int attn_get_last_device_error(void* stream, unsigned int* detail) {
@@ -716,6 +904,13 @@ int attn_get_last_device_error(void* stream, unsigned int* detail) {
     return ATTN_ERR_CUDA;
   if (detail != nullptr) *detail = word;
   return word != 0 ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
+}
+
+int attn_debug_map_cache_stats(unsigned long long* hits, unsigned long long* encodes) {
+  if (hits == nullptr || encodes == nullptr) return ATTN_ERR_INVALID_ARG;
+  *hits = g_map_hits.load(std::memory_order_relaxed);
+  *encodes = g_map_encodes.load(std::memory_order_relaxed);
+  return ATTN_OK;
 }
 
 int attn_debug_exp2(const float* x, float* y, long long n, int mode, void* stream) {

@@ -14,8 +14,12 @@ struct FwdParams {
   float* lse;       // [B, Hq, Nq] fp32 or nullptr
   int B, Hq, Hkv, Nq, Nk;
   int group;        // Hq / Hkv
+  // the part of the problem this launch computes: batches [b0, b0 + nb) and
+  // query heads [h0, h0 + nh) (whole key/value groups); the tensors above are
+  // the full [B, N, H, d] ones
+  int b0, nb, h0, nh;
   int n_qblocks;    // ceil(Nq / (128 * NQT))
-  int n_items;      // B * Hq * n_qblocks work items
+  int n_items;      // nb * nh * n_qblocks work items
   int qb_major;     // 1: order items by query block (longest first) across heads; 0: head-major
   float sl2;        // scale * log2(e)
   // split-KV (one-block-per-item kernel): the keys are cut into n_splits
@@ -179,6 +183,28 @@ template <int ROLE = 0>
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const WaitCtx& c, uint32_t site) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   return wait_bar_slow<ROLE>(bar, parity, c, site);
+}
+
+// Drain wait of a producer before its block exits: a TMA copy that was issued
+// lands whether or not anything consumes it, so this wait ignores the block's
+// abort flag (the block must not free its shared memory under a copy in
+// flight) and ends only when the phase completes or the time limit passes.
+template <int ROLE>
+__device__ __noinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity, const WaitCtx& c, uint32_t site) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (ptx::mbar_try_wait(bar, parity)) return true;
+    if constexpr (ROLE == kRoleProducerBackoff) __nanosleep(64);
+    if (ptx::globaltimer() - t0 > c.timeout_ns) {
+      *c.abort = 1u;
+      const uint32_t blk = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+      atomicOr(c.err, 1u | (site << 8) | ((blk & 0xFFFFu) << 16));
+      return false;
+    }
+  }
 }
 
 // Wait by a whole warp (every lane polls the same barrier); the result is made

@@ -80,8 +80,9 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = p.n_qblocks - 1 - (int)blockIdx.x;  // longest causal blocks first
   const int g = Cfg::PACK ? p.pack : 1;  // query heads stacked per tile row group
-  const int hy = blockIdx.y;         // query head, or key/value head when packed
-  const int b = (int)blockIdx.z / p.n_splits, split = (int)blockIdx.z % p.n_splits;
+  // query head, or key/value head when packed (grid y covers the launch's heads)
+  const int hy = (g > 1 ? p.h0 / g : p.h0) + (int)blockIdx.y;
+  const int b = p.b0 + (int)blockIdx.z / p.n_splits, split = (int)blockIdx.z % p.n_splits;
   // key window of this block: [kv0, kv0 + nk), `shift` keys after it
   const int kv0 = split * p.kv_chunk;
   const int nk = p.Nk - kv0 < p.kv_chunk ? p.Nk - kv0 : p.kv_chunk;
@@ -405,13 +406,13 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       // normal path, where the consumers have already seen them all).
 #pragma unroll
       for (int t = 0; t < NQT; ++t)
-        if (q_issued[t]) wait_bar<kRoleProducer>(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
+        if (q_issued[t]) wait_bar_drain<kRoleProducer>(bar(Cfg::B_QFULL + t), 0u, wc, kSiteQ);
 #pragma unroll
       for (int s = 0; s < KST; ++s)
-        if (k_issued[s] > 0) wait_bar<kRoleProducer>(bar(Cfg::B_KFULL + s), (uint32_t)((k_issued[s] - 1) & 1), wc, kSiteKFull);
+        if (k_issued[s] > 0) wait_bar_drain<kRoleProducer>(bar(Cfg::B_KFULL + s), (uint32_t)((k_issued[s] - 1) & 1), wc, kSiteKFull);
 #pragma unroll
       for (int s = 0; s < VST; ++s)
-        if (v_issued[s] > 0) wait_bar<kRoleProducer>(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
+        if (v_issued[s] > 0) wait_bar_drain<kRoleProducer>(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
     }
   } else {
     if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_dec<Cfg::REG_CONTROL>();

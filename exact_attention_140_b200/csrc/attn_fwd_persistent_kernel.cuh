@@ -59,7 +59,7 @@ struct Item {
   int qb, h, b;
 };
 __device__ __forceinline__ Item decode_item(int i, const FwdParams& p) {
-  const int bh = p.B * p.Hq;
+  const int bh = p.nb * p.nh;
   int qr, r;
   if (p.qb_major) {
     qr = i / bh;
@@ -68,7 +68,7 @@ __device__ __forceinline__ Item decode_item(int i, const FwdParams& p) {
     r = i / p.n_qblocks;
     qr = i - r * p.n_qblocks;
   }
-  return Item{p.n_qblocks - 1 - qr, r % p.Hq, r / p.Hq};
+  return Item{p.n_qblocks - 1 - qr, p.h0 + r % p.nh, p.b0 + r / p.nh};
 }
 
 template <class Cfg>
@@ -462,15 +462,15 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
 #pragma unroll
       for (int t = 0; t < NQT; ++t)
         if (q_issued[t] > 0)
-          wait_bar<kProducerRole>(bar(Cfg::B_QFULL + t), (uint32_t)((q_issued[t] - 1) & 1), wc, kSiteQ);
+          wait_bar_drain<kProducerRole>(bar(Cfg::B_QFULL + t), (uint32_t)((q_issued[t] - 1) & 1), wc, kSiteQ);
 #pragma unroll
       for (int s = 0; s < KST; ++s)
         if (k_issued[s] > 0)
-          wait_bar<kProducerRole>(bar(Cfg::B_KFULL + s), (uint32_t)((k_issued[s] - 1) & 1), wc, kSiteKFull);
+          wait_bar_drain<kProducerRole>(bar(Cfg::B_KFULL + s), (uint32_t)((k_issued[s] - 1) & 1), wc, kSiteKFull);
 #pragma unroll
       for (int s = 0; s < VST; ++s)
         if (v_issued[s] > 0)
-          wait_bar<kProducerRole>(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
+          wait_bar_drain<kProducerRole>(bar(Cfg::B_VFULL + s), (uint32_t)((v_issued[s] - 1) & 1), wc, kSiteVFull);
     }
   } else {
     if constexpr (Cfg::SPLIT_REGS) ptx::setmaxnreg_dec<Cfg::REG_CONTROL>();

@@ -4,96 +4,240 @@
 // the per-tensor absolute maximum, and quantise to E4M3 with
 // descale = amax / 448.
 //
-// One warp owns one row of d = 128 elements, 4 consecutive elements per
-// lane.  The rotation is a fast Walsh-Hadamard transform: butterflies of
-// span 1 and 2 inside a lane, spans 4..64 across lanes with shuffles.  Two
-// passes over the input (HBM-bound): pass 1 finds amax, pass 2 rotates again
-// and writes the codes (recomputing the transform costs less than a round
-// trip of the rotated tensor through HBM).
+// HBM-bound (2 bytes read and 1 byte written per element), so the design is
+// about bytes in flight and few instructions per element:
+//   * tiles of 128 rows x 128 columns (32 KB of bf16) are brought into shared
+//     memory by TMA (two 128-byte-wide boxes, 128-byte swizzle) through a
+//     ring of stages, several tiles ahead of the compute;
+//   * thread t of a 128-thread block owns row t of the tile: it reads the row
+//     from shared memory (the swizzle spreads the 16-byte chunks of eight
+//     consecutive rows over all banks, so the reads are conflict-free), and
+//     runs the whole fast Walsh-Hadamard transform in registers (level 0 in
+//     scalar fp32, levels 1-6 as packed fp32x2 butterflies) -- no shuffles;
+//   * the random signs are applied as XOR masks on the bf16 sign bits before
+//     the values are widened (an exact multiplication by +-1), and 1/sqrt(d)
+//     is folded into the final scale: fl(max|y| * c) = max fl(|y| * c) for
+//     c > 0, so amax is what scaling every value first would give;
+//   * the quantising pass writes each row's 128 codes into a swizzled
+//     shared-memory tile that one TMA store writes back; rows past the end of
+//     the tensor are zero-filled on load and clipped on store.
+// Two passes (amax, then quantise) because every code depends on the global
+// amax; the second pass walks the tiles in reverse order, so it starts on the
+// ones the first pass read last, which are the likeliest to be in L2.
 #pragma once
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "attn_common.cuh"
 #include "ptx.cuh"
 
 namespace attn {
 
 constexpr int kPrepD = 128;
-constexpr int kPrepWarps = 8;
+constexpr int kPrepRows = 128;                               // rows per tile = threads per block
+constexpr uint32_t kPrepHalfBytes = kPrepRows * 128;         // one 64-column box of bf16
+constexpr uint32_t kPrepTileBytes = 2 * kPrepHalfBytes;      // 32 KB
+constexpr uint32_t kPrepOutBytes = kPrepRows * kPrepD;       // 16 KB of codes
+constexpr float kPrepInvSqrtD = 0.08838834764831845f;        // 1/sqrt(128)
 
-// Loads row r (4 values per lane), applies signs and the transform when
-// `signs` is not null.  Returns the lane's 4 rotated values.
-__device__ __forceinline__ void prep_row(const __nv_bfloat16* __restrict__ x, long long r,
-                                         const float* __restrict__ signs, float (&v)[4]) {
-  const int lane = threadIdx.x & 31;
-  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(x + r * kPrepD) + lane);
-  v[0] = __uint_as_float(raw.x << 16);
-  v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-  v[2] = __uint_as_float(raw.y << 16);
-  v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-  if (signs == nullptr) return;
-  const float4 s = __ldg(reinterpret_cast<const float4*>(signs) + lane);
-  v[0] *= s.x;
-  v[1] *= s.y;
-  v[2] *= s.z;
-  v[3] *= s.w;
-  // span 1 and span 2 inside the lane (element index 4*lane + e)
-  float a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
-  v[0] = a0 + a2;
-  v[1] = a1 + a3;
-  v[2] = a0 - a2;
-  v[3] = a1 - a3;
-  // spans 4, 8, 16, 32, 64 = lane distances 1, 2, 4, 8, 16
+template <bool QUANT>
+struct PrepCfg {
+  static constexpr int STAGES = QUANT ? 2 : 3;
+  static constexpr uint32_t OFF_IN = 0;
+  static constexpr uint32_t OFF_OUT = STAGES * kPrepTileBytes;
+  static constexpr uint32_t OFF_BAR = OFF_OUT + (QUANT ? kPrepOutBytes : 0);
+  // the sign masks are read as 16-byte vectors: 16-byte aligned
+  static constexpr uint32_t OFF_MASK = (OFF_BAR + 8 * STAGES + 15u) & ~15u;
+  static constexpr uint32_t OFF_ABORT = OFF_MASK + 64 * 4;
+  static constexpr uint32_t OFF_RED = OFF_ABORT + 16;
+  static constexpr uint32_t SMEM_BYTES = OFF_RED + 4 * 4 + 1024;  // + alignment slack
+  static_assert(OFF_MASK % 16 == 0 && OFF_IN % 1024 == 0 && OFF_OUT % 1024 == 0, "vector and TMA alignment");
+  static_assert(2 * SMEM_BYTES <= 227 * 1024, "two blocks per SM");
+};
+
+struct PrepParams {
+  long long rows;
+  int n_tiles;
+  const float* signs;        // d values, +1 or -1; nullptr: no rotation
+  unsigned int* amax_bits;   // running max of |rotated value| as float bits
+  float* descale;            // amax / 448 (quantising pass)
+  unsigned int* err;
+  unsigned long long timeout_ns;
+};
+
+// Row t of the tile in stage memory `tile` (two swizzled 64-column boxes) ->
+// 128 fp32 values, signs applied (XOR masks on the bf16 sign bits), then the
+// unnormalised Walsh-Hadamard transform when ROT.  v[2k], v[2k+1] live in
+// one packed register pair P[k].
+template <bool ROT>
+__device__ __forceinline__ void prep_load_transform(const uint8_t* tile, const uint4* mask4, int r,
+                                                    uint64_t (&P)[64]) {
 #pragma unroll
-  for (int ld = 1; ld < 32; ld <<= 1) {
-    const bool upper = (lane & ld) != 0;
+  for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float w = __shfl_xor_sync(0xffffffffu, v[e], ld);
-      v[e] = upper ? (w - v[e]) : (v[e] + w);
+    for (int c = 0; c < 8; ++c) {
+      uint4 w = *reinterpret_cast<const uint4*>(tile + h * kPrepHalfBytes + r * 128 + ((c ^ (r & 7)) << 4));
+      if constexpr (ROT) {
+        const uint4 m = mask4[h * 8 + c];
+        w.x ^= m.x;
+        w.y ^= m.y;
+        w.z ^= m.z;
+        w.w ^= m.w;
+      }
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xFFFF0000u);
+        if constexpr (ROT) {
+          // level 0 of the transform (span 1) on the pair as it is widened
+          P[h * 32 + c * 4 + e] = ptx::f2(lo + hi, lo - hi);
+        } else {
+          P[h * 32 + c * 4 + e] = ptx::f2(lo, hi);
+        }
+      }
+    }
+  if constexpr (ROT) {
+    // levels 1..6 (spans 2..64 elements = 1..32 pairs): packed butterflies
+#pragma unroll
+    for (int sp = 1; sp < 64; sp <<= 1)
+#pragma unroll
+      for (int k = 0; k < 64; ++k)
+        if ((k & sp) == 0) {
+          const uint64_t a = P[k], b = P[k + sp];
+          P[k] = ptx::fadd2(a, b);
+          P[k + sp] = ptx::fsub2(a, b);
+        }
+  }
+}
+
+// One pass over the tensor: QUANT = false accumulates amax (one atomicMax per
+// block), QUANT = true writes the codes and, from block 0, the descale.
+template <bool ROT, bool QUANT>
+__global__ void __launch_bounds__(kPrepRows, 2)
+    fp8_prep_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmX8,
+                    const PrepParams p) {
+  using C = PrepCfg<QUANT>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
+  const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw_u32);
+  auto bar = [&](int s) -> uint32_t { return sbase + C::OFF_BAR + 8u * (uint32_t)s; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sgen + C::OFF_ABORT);
+  const WaitCtx wc{abort_flag, p.err, p.timeout_ns};
+  const int tid = threadIdx.x;
+  const int G = (int)gridDim.x;
+  // tile of this block's k-th step (the quantising pass walks them backwards)
+  auto tile_at = [&](int k) -> int {
+    const long long i = (long long)blockIdx.x + (long long)k * G;
+    if (i >= p.n_tiles) return -1;
+    return QUANT ? p.n_tiles - 1 - (int)i : (int)i;
+  };
+
+  uint32_t* mask = reinterpret_cast<uint32_t*>(sgen + C::OFF_MASK);
+  if (tid < 64) {
+    uint32_t m = 0u;
+    if (ROT) {
+      if (__ldg(p.signs + 2 * tid) < 0.f) m |= 0x00008000u;
+      if (__ldg(p.signs + 2 * tid + 1) < 0.f) m |= 0x80000000u;
+    }
+    mask[tid] = m;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) ptx::mbar_init(bar(s), 1);
+    *abort_flag = 0u;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmX);
+    if (QUANT) ptx::prefetch_tmap(&tmX8);
+  }
+  __syncthreads();
+
+  int issued[C::STAGES];
+#pragma unroll
+  for (int s = 0; s < C::STAGES; ++s) issued[s] = 0;
+  auto issue = [&](int k) {  // thread 0: load the tile of step k into stage k % STAGES
+    const int tile = tile_at(k);
+    if (tile < 0) return;
+    const int s = k % C::STAGES;
+    const uint32_t dst = sbase + C::OFF_IN + (uint32_t)s * kPrepTileBytes;
+    ptx::mbar_arrive_expect_tx(bar(s), kPrepTileBytes);
+    ptx::tma_load_2d(dst, &tmX, bar(s), 0, tile * kPrepRows);
+    ptx::tma_load_2d(dst + kPrepHalfBytes, &tmX, bar(s), 64, tile * kPrepRows);
+    ++issued[s];
+  };
+  if (tid == 0)
+    for (int k = 0; k < C::STAGES; ++k) issue(k);
+
+  float mult = 0.f;
+  if constexpr (QUANT) {
+    const float amax = __uint_as_float(*p.amax_bits);
+    const float inv = amax > 0.f ? 448.0f / amax : 0.f;
+    mult = ROT ? kPrepInvSqrtD * inv : inv;
+    if (blockIdx.x == 0 && tid == 0) *p.descale = amax > 0.f ? amax / 448.0f : 1.0f;
+  }
+  const uint4* mask4 = reinterpret_cast<const uint4*>(mask);
+  float m0 = 0.f, m1 = 0.f;
+  for (int k = 0;; ++k) {
+    const int tile = tile_at(k);
+    if (tile < 0) break;
+    const int s = k % C::STAGES;
+    bool ok = wait_bar<kRoleSoftmax>(bar(s), (uint32_t)((k / C::STAGES) & 1), wc, kSiteKFull);
+    uint64_t P[64];
+    if (ok) prep_load_transform<ROT>(sgen + C::OFF_IN + (uint32_t)s * kPrepTileBytes, mask4, tid, P);
+    if constexpr (QUANT) {
+      if (tid == 0) ptx::bulk_wait_read0();  // the previous tile's store has read the output buffer
+    }
+    if (!__syncthreads_and(ok)) break;  // stage s is consumed by every thread
+    if (tid == 0) issue(k + C::STAGES);
+    if constexpr (!QUANT) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        float a, b;
+        ptx::unf2(P[i], a, b);
+        m0 = fmaxf(m0, fabsf(a));
+        m1 = fmaxf(m1, fabsf(b));
+      }
+    } else {
+      uint8_t* out = sgen + C::OFF_OUT;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {  // 16 codes (one 16-byte chunk) at a time
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float a, b, cc, d;
+          ptx::unf2(P[c * 8 + 2 * e], a, b);
+          ptx::unf2(P[c * 8 + 2 * e + 1], cc, d);
+          w[e] = ptx::pack_e4m3x4(a * mult, b * mult, cc * mult, d * mult);
+        }
+        *reinterpret_cast<uint4*>(out + tid * 128 + ((c ^ (tid & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      ptx::fence_proxy_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        ptx::tma_store_2d(&tmX8, sbase + C::OFF_OUT, 0, tile * kPrepRows);
+        ptx::bulk_commit();
+      }
     }
   }
-  const float inv_sqrt_d = 0.08838834764831845f;  // 1/sqrt(128)
+  if (tid == 0) {
+    // every issued load must land and every store must finish before exit
 #pragma unroll
-  for (int e = 0; e < 4; ++e) v[e] *= inv_sqrt_d;
-}
-
-__global__ void __launch_bounds__(32 * kPrepWarps) fp8_amax_kernel(const __nv_bfloat16* __restrict__ x, long long rows,
-                                                                     const float* __restrict__ signs,
-                                                                     unsigned int* __restrict__ amax_bits) {
-  __shared__ float red[kPrepWarps];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float m = 0.f;
-  for (long long r = (long long)blockIdx.x * kPrepWarps + warp; r < rows; r += (long long)gridDim.x * kPrepWarps) {
-    float v[4];
-    prep_row(x, r, signs, v);
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+    for (int s = 0; s < C::STAGES; ++s)
+      if (issued[s] > 0) wait_bar_drain<kRoleProducer>(bar(s), (uint32_t)((issued[s] - 1) & 1), wc, kSiteDrain);
+    if (QUANT) ptx::bulk_wait0();
   }
+  if constexpr (!QUANT) {
+    float m = fmaxf(m0, m1);
+    if (ROT) m *= kPrepInvSqrtD;  // monotone: the max of the scaled values
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[warp] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float bm = red[0];
-    for (int w = 1; w < kPrepWarps; ++w) bm = fmaxf(bm, red[w]);
-    atomicMax(amax_bits, __float_as_uint(bm));  // non-negative floats order like their bits
-  }
-}
-
-__global__ void __launch_bounds__(32 * kPrepWarps) fp8_quant_kernel(const __nv_bfloat16* __restrict__ x, long long rows,
-                                                                      const float* __restrict__ signs,
-                                                                      const unsigned int* __restrict__ amax_bits,
-                                                                      uint8_t* __restrict__ x8,
-                                                                      float* __restrict__ descale) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float amax = __uint_as_float(*amax_bits);
-  const float inv = amax > 0.f ? 448.0f / amax : 0.f;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *descale = amax > 0.f ? amax / 448.0f : 1.0f;
-  for (long long r = (long long)blockIdx.x * kPrepWarps + warp; r < rows; r += (long long)gridDim.x * kPrepWarps) {
-    float v[4];
-    prep_row(x, r, signs, v);
-    const uint32_t codes = ptx::pack_e4m3x4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
-    reinterpret_cast<uint32_t*>(x8 + r * kPrepD)[lane] = codes;
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float* red = reinterpret_cast<float*>(sgen + C::OFF_RED);
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    __syncthreads();
+    if (tid == 0) {
+      const float bm = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+      atomicMax(p.amax_bits, __float_as_uint(bm));  // non-negative floats order like their bits
+    }
   }
 }
 

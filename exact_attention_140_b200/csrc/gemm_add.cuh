@@ -117,7 +117,9 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
       const long long row_off = (long long)row * p.N;
       // C does not depend on the products: this thread's 128 values of it are
       // requested before the accumulator is waited for, so the loads overlap
-      // the wait and each other (N is a multiple of 8: 8-column groups are whole)
+      // the wait and each other (N is a multiple of 8: 8-column groups are whole).
+      // Plain (coherent) loads: C may be D itself (an in-place update), and the
+      // thread that reads an element of C is the one that later writes it to D.
       uint4 cr[4][4];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
         for (int g = 0; g < 4; ++g) {
           const int col = n0 + wg * 128 + 32 * c + 8 * g;
           cr[c][g] = (p.c != nullptr && row_ok && col < p.N)
-                         ? __ldg(reinterpret_cast<const uint4*>(p.c + row_off + col))
+                         ? *reinterpret_cast<const uint4*>(p.c + row_off + col)
                          : make_uint4(0u, 0u, 0u, 0u);
         }
       ok = wait_bar<kRoleSoftmax>(bar(G::B_ACCF + acc), (uint32_t)((k >> 1) & 1), wc, kSiteODone);
@@ -197,7 +199,7 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
 #pragma unroll
       for (int s = 0; s < G::STAGES; ++s)
         if (issued[s] > 0)
-          wait_bar<kRoleProducer>(bar(G::B_FULL + s), (uint32_t)((issued[s] - 1) & 1), wc, kSiteKFull);
+          wait_bar_drain<kRoleProducer>(bar(G::B_FULL + s), (uint32_t)((issued[s] - 1) & 1), wc, kSiteKFull);
     }
   } else if (warp == G::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer

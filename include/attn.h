@@ -80,6 +80,41 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
              int dtype, void *stream);
 
 /*
+ * attn_fwd_part -- attn_fwd restricted to batches [b_begin, b_end) and the
+ * query heads of key/value heads [kvh_begin, kvh_end) (query heads
+ * [kvh_begin * g, kvh_end * g) with g = Hq / Hkv, so a grouped-query group is
+ * never split).  Every (batch, head) of the problem is independent (page
+ * "FlashAttention (SV)", the attention formula is applied per head), so
+ * several devices can each compute a part of one call on the same full
+ * tensors, with no exchange of data between them.
+ *   q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype, stream
+ *                as attn_fwd: the FULL tensors and sizes of the call
+ *   b_begin, b_end      0 <= b_begin <= b_end <= B
+ *   kvh_begin, kvh_end  0 <= kvh_begin <= kvh_end <= Hkv
+ * Only the O rows and LSE entries of the part are written; the rest of o and
+ * lse is left as it was.  An empty range is a no-op.  attn_fwd is this call
+ * with the whole range.  Returns ATTN_ERR_INVALID_ARG for a range outside the
+ * problem; otherwise as attn_fwd.
+ */
+int attn_fwd_part(const void *q, const void *k, const void *v, void *o, float *lse,
+                  int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                  int dtype, int b_begin, int b_end, int kvh_begin, int kvh_end, void *stream);
+
+/*
+ * attn_shard_units -- the share of one call that rank `rank` of `world`
+ * computes when the call is split over devices: the B * Hkv units (batch,
+ * key/value head) are cut in batch-major order into `world` contiguous runs
+ * whose lengths differ by at most one; rank r takes run r.  The run is
+ * written to rects as up to three rectangles, rectangle i being
+ * rects[4i .. 4i+3] = {b_begin, b_end, kvh_begin, kvh_end}, each one
+ * attn_fwd_part call (rects must hold 12 ints).  Returns the number of
+ * rectangles (0 when the rank has no unit), or -1 for invalid arguments
+ * (B < 0, Hkv < 0, world < 1, rank outside [0, world), rects NULL).
+ * Host-only; no CUDA call.
+ */
+int attn_shard_units(int B, int Hkv, int world, int rank, int *rects);
+
+/*
  * attn_fwd_fp8 -- FP8 E4M3 attention forward with per-tensor scales.
  * Page "FlashAttention-3 — 闪电注意力-3", section 3: the inputs are quantised
  * (Q and K after the Hadamard rotation, see attn_hadamard_quant_fp8) and the
@@ -238,9 +273,13 @@ int attn_tile_kind_window(int row0, int row1, int kt, int Nq, int Nk, int shift,
  *   a  [M, K] bf16, b [K, N] bf16, c [M, N] bf16 or NULL (no addition),
  *   d  [M, N] bf16 output; all row-major DEVICE pointers, 16-byte aligned.
  * Products accumulate in fp32; D = bf16(A B + C), round to nearest even.
- * N and K must be multiples of 8 (ATTN_ERR_UNSUPPORTED otherwise); K = 0
- * gives D = C (or 0).  Any M and N; any K, though the design targets small K
- * (the kernel is then HBM-bound on reading C and writing D).
+ * Sizes: any M >= 0; N and K multiples of 8 (ATTN_ERR_UNSUPPORTED
+ * otherwise), with the row strides 2N and 2K bytes and the matrix extents
+ * within the Tensor Memory Accelerator's limits (ATTN_ERR_CUDA when a tensor
+ * map cannot be encoded).  K = 0 gives D = C (or 0).  The design targets
+ * small K (the kernel is then HBM-bound on reading C and writing D).
+ * Aliasing: c == d is allowed (an in-place D += A B); a c that overlaps d
+ * any other way returns ATTN_ERR_INVALID_ARG.  a and b must not overlap d.
  */
 int attn_gemm_add(const void *a, const void *b, const void *c, void *d, int M, int N, int K, void *stream);
 
@@ -262,6 +301,17 @@ int attn_fwd_schedule(int Nk);
  * finish ends with an error status and leaves the context usable.
  */
 int attn_debug_unsatisfied_wait(long long limit_ns, void *stream);
+
+/*
+ * Counters of the library's tensor-map cache (host only, never fails for
+ * non-NULL arguments): `hits` counts tensor maps taken from the cache,
+ * `encodes` those encoded afresh.  Every launch needs one map per Q/K/V
+ * operand (A/B for attn_gemm_add); a map is a pure function of the tensor's
+ * base address, shape and tile box, so calls that reuse the same tensors skip
+ * the encoding.  The cache holds 256 maps (64 sets of 4) and is guarded by a
+ * mutex.
+ */
+int attn_debug_map_cache_stats(unsigned long long *hits, unsigned long long *encodes);
 
 /*
  * Debug hook for the softmax exponential: y[i] = 2^x[i] for n values, as the

@@ -59,14 +59,16 @@ def bf16_ulp(x):
 def compare(o, lse, o_ref, lse_ref, tol=BF16_TOL):
     """Elementwise comparison with the stated tolerances; rows the oracle marks
     empty (LSE = -inf) must be exactly O = 0 and LSE = -inf.  The max bound is
-    1e-2, or one bf16 ulp of the exact value where that is larger (|O| >= 4,
-    where rounding the output to bf16 alone can exceed 1e-2).  Likewise the
-    mean bound is 1e-3, or half the mean bf16 ulp of the exact values where
+    1e-2, or, where larger, what bf16 arithmetic alone can cost at that output:
+    the final rounding of O (half a bf16 ulp of the exact value) plus P rounded
+    to bf16 before P V (relative 2^-9 per weight; |O| above ~2.5 only occurs in
+    rows dominated by a few keys, where it moves O by up to 2^-9 |O|).  Likewise
+    the mean bound is 1e-3, or half the mean bf16 ulp of the exact values where
     that is larger: for outputs of a handful of keys (|O| ~ 1) exact rounding
     to bf16 alone has a mean error near ulp/4 ~ 2e-3."""
     assert np.all(np.isfinite(o)), "non-finite output"
     err = np.abs(o - o_ref)
-    bound = np.maximum(tol["max_abs"], bf16_ulp(o_ref))
+    bound = np.maximum(tol["max_abs"], 0.5 * bf16_ulp(o_ref) + 2.0 ** -9 * np.abs(o_ref))
     worst = np.argmax(err - bound)
     assert err.flat[worst] <= bound.flat[worst], f"|dO| = {err.flat[worst]:.3g} > {bound.flat[worst]:.3g}"
     mean_bound = max(tol["mean_abs"], 0.5 * float(np.mean(bf16_ulp(o_ref))))

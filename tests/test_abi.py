@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import exact_attention_140_b200 as ea
@@ -156,3 +157,70 @@ def test_gemm_add_argument_errors_before_any_cuda_call():
     assert g(a=FAKE + 8) == MISALIGNED
     assert g(c=FAKE + 2) == MISALIGNED
     assert g(M=0) == OK and g(N=0) == OK
+
+
+def test_gemm_add_partial_overlap_of_c_and_d_rejected():
+    """C may be D itself (an in-place update) but may not partly overlap it:
+    another thread's store to D could then land before C is read."""
+    def g(c, d, M=128, N=256):
+        return ea.attn_gemm_add(FAKE, FAKE, c, d, M, N, 64, stream=0, raise_on_error=False)
+    nbytes = 128 * 256 * 2
+    assert g(FAKE + 16, FAKE) == INVALID
+    assert g(FAKE, FAKE + nbytes - 16) == INVALID
+    # disjoint ranges and the exact alias pass the argument checks (and then
+    # fail only for want of a GPU here)
+    assert g(FAKE + nbytes, FAKE) != INVALID
+    assert g(FAKE, FAKE) != INVALID
+
+
+@pytest.mark.parametrize("B,Hkv", [(1, 1), (2, 8), (3, 5), (4, 1), (7, 3), (1, 16), (0, 4)])
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_shard_units_cover_every_unit_once(B, Hkv, world):
+    """The B x Hkv (batch, key/value head) units of one call split over `world`
+    ranks: every unit belongs to exactly one rank, the ranks' shares differ by
+    at most one unit, and each rank's share is a contiguous batch-major run."""
+    owner = np.full((B, Hkv), -1)
+    sizes = []
+    for r in range(world):
+        rects = ea.attn_shard_units(B, Hkv, world, r)
+        assert len(rects) <= 3
+        units = []
+        for (b0, b1, g0, g1) in rects:
+            assert 0 <= b0 < b1 <= B and 0 <= g0 < g1 <= Hkv
+            assert np.all(owner[b0:b1, g0:g1] == -1)
+            owner[b0:b1, g0:g1] = r
+            units += [b * Hkv + g for b in range(b0, b1) for g in range(g0, g1)]
+        units.sort()
+        if units:
+            assert units == list(range(units[0], units[-1] + 1))
+        sizes.append(len(units))
+    assert np.all(owner >= 0)
+    assert max(sizes) - min(sizes) <= 1
+    # ranks in order: rank r's run precedes rank r+1's
+    firsts = [min((b * Hkv + g for b, g in zip(*np.nonzero(owner == r))), default=None) for r in range(world)]
+    got = [f for f in firsts if f is not None]
+    assert got == sorted(got)
+
+
+def test_shard_units_invalid():
+    with pytest.raises(ea.AttnError):
+        ea.attn_shard_units(2, 2, 0, 0)
+    with pytest.raises(ea.AttnError):
+        ea.attn_shard_units(2, 2, 2, 2)
+    with pytest.raises(ea.AttnError):
+        ea.attn_shard_units(-1, 2, 2, 0)
+
+
+def test_fwd_part_range_errors_before_any_cuda_call():
+    def part(b0, b1, g0, g1, **kw):
+        a = dict(B=2, Hq=8, Hkv=4, Nq=64, Nk=64, d=128)
+        a.update(kw)
+        return ea.attn_fwd_part(FAKE, FAKE, FAKE, FAKE, None, a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"], a["d"],
+                                0, 0.1, ea.ATTN_BF16, b0, b1, g0, g1, stream=0, raise_on_error=False)
+    assert part(-1, 1, 0, 4) == INVALID
+    assert part(1, 0, 0, 4) == INVALID
+    assert part(0, 3, 0, 4) == INVALID
+    assert part(0, 2, 2, 1) == INVALID
+    assert part(0, 2, 0, 5) == INVALID
+    assert part(0, 2, 0, 4, d=96) == UNSUPPORTED
+    assert part(0, 2, 0, 4, Nq=0) == OK  # nothing to compute

@@ -3,6 +3,7 @@ output is computed on the GPU and sampled rows are recomputed one by one by
 the fp64 oracle; every output must be finite and every LSE finite (no empty
 rows at Nq == Nk)."""
 import math
+import zlib
 
 import numpy as np
 import pytest
@@ -43,7 +44,7 @@ def test_fullsize_sampled_rows(name):
     scale = 1.0 / math.sqrt(d)
     o, lse = run_attn(qb, kb, vb, causal, scale)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
-    rows = sample_rows(B, Hq, N, np.random.default_rng(hash(name) % 1000))
+    rows = sample_rows(B, Hq, N, np.random.default_rng(zlib.crc32(name.encode())))
     o_ref, lse_ref = oracle.attn_fwd_rows(gen.bf16_bits_to_f64(qb), gen.bf16_bits_to_f64(kb),
                                           gen.bf16_bits_to_f64(vb), causal, scale, rows)
     b, h, i = rows // (Hq * N), (rows // N) % Hq, rows % N

@@ -73,3 +73,20 @@ def test_bench_shape_sampled_rows():
     acc = K * 2.0 ** -23 * oracle.gemm_add(np.abs(a64), np.abs(b64), np.abs(c64))
     err = np.abs(d[rows] - ref)
     assert np.all(err <= bf16_ulp(ref) + acc)
+
+
+def test_in_place_c_is_d():
+    """c == d: D += A B in place (each epilogue thread reads its C elements
+    before it stores the same elements of D)."""
+    import exact_attention_140_b200 as ea
+    M, N, K = 300, 520, 64
+    ab, bb, cb = gen.normal_bf16(21, (M, K)), gen.normal_bf16(22, (K, N)), gen.normal_bf16(23, (M, N))
+    T = torch_mod()
+    a, b, cd = to_dev_bf16(ab), to_dev_bf16(bb), to_dev_bf16(cb)
+    ea.attn_gemm_add(a, b, cd, cd, M, N, K)
+    rc, word = ea.attn_get_last_device_error()
+    assert rc == 0, hex(word)
+    got = bf16_dev_to_f64(cd)
+    ref_out = run_gemm(ab, bb, cb)  # the same product into a separate D
+    assert np.array_equal(got, ref_out)
+    T.cuda.synchronize()

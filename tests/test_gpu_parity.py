@@ -186,3 +186,13 @@ def test_repeatable(N):
     a = run_attn(qb, kb, vb, True)
     b = run_attn(qb, kb, vb, True)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# A negative scale turns the row maximum of the raw scores into the row
+# minimum (a separate branch in both kernels); full and diagonal tiles, on the
+# persistent kernel (key ranges <= 1024) and the one-block-per-item kernel.
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("N", [300, 1100])
+@pytest.mark.parametrize("causal", [False, True])
+def test_negative_scale(d, N, causal):
+    full_check(1, 2, 1, N, N, d, causal, scale=-1.0 / math.sqrt(d))

@@ -70,3 +70,56 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
     args = type("A", (), dict(steps=1, warmup=0, gpus=2, cpu_seconds=1.0))()
     assert bench.run_reference(args, bench.workloads()["tiny"], "tiny") == 0
     assert capsys.readouterr().out == ""
+
+
+def _shard_worker(rank, world, port, out_dir):
+    """One rank of a call split by (batch, key/value head) units: it computes its
+    rectangles (the oracle stands in for the GPU here) and the pieces are
+    gathered to rank 0 over gloo, which reassembles the whole output."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    import attn_inputs as gen
+    import exact_attention_140_b200 as ea
+    import oracle
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    B, Hq, Hkv, N, d = 3, 6, 3, 24, 8
+    g = Hq // Hkv
+    q, k, v = (gen.bf16_bits_to_f64(x) for x in gen.qkv_bf16(B, Hq, Hkv, N, N, d, seed=91))
+    pieces = []
+    for (b0, b1, g0, g1) in ea.attn_shard_units(B, Hkv, world, rank):
+        o, lse = oracle.attn_fwd(q[b0:b1, :, g0 * g:g1 * g], k[b0:b1, :, g0:g1], v[b0:b1, :, g0:g1], True, 0.3)
+        pieces.append(((b0, b1, g0, g1), o, lse))
+    gathered = [None] * world
+    dist.all_gather_object(gathered, pieces)
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank == 0:
+        o_all = np.full((B, N, Hq, d), np.nan)
+        lse_all = np.full((B, Hq, N), np.nan)
+        for rank_pieces in gathered:
+            for (b0, b1, g0, g1), o, lse in rank_pieces:
+                assert np.all(np.isnan(o_all[b0:b1, :, g0 * g:g1 * g]))  # no unit computed twice
+                o_all[b0:b1, :, g0 * g:g1 * g] = o
+                lse_all[b0:b1, g0 * g:g1 * g] = lse
+        o_ref, lse_ref = oracle.attn_fwd(q, k, v, True, 0.3)
+        np.save(os.path.join(out_dir, "o_all.npy"), o_all)
+        np.save(os.path.join(out_dir, "o_ref.npy"), o_ref)
+        np.save(os.path.join(out_dir, "lse_all.npy"), lse_all)
+        np.save(os.path.join(out_dir, "lse_ref.npy"), lse_ref)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_call_reassembles_on_gloo_ranks(tmp_path, world):
+    import torch.multiprocessing as mp
+    port = _free_port()
+    mp.start_processes(_shard_worker, args=(world, port, str(tmp_path)), nprocs=world, start_method="spawn",
+                       join=True)
+    o_all, o_ref = np.load(tmp_path / "o_all.npy"), np.load(tmp_path / "o_ref.npy")
+    lse_all, lse_ref = np.load(tmp_path / "lse_all.npy"), np.load(tmp_path / "lse_ref.npy")
+    assert not np.isnan(o_all).any()  # every unit computed by some rank
+    assert np.array_equal(o_all, o_ref) and np.array_equal(lse_all, lse_ref)

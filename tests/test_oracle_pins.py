@@ -304,3 +304,35 @@ def test_generator_is_seeded_and_standard_normal():
     bits = gen.f32_to_bf16_bits(np.array([1.0, 1.00390625, 1.01171875, -2.5], dtype=np.float32))
     # 1.00390625 = 1 + 2^-8 is a tie between bf16 1.0 and 1.0078125 -> even (1.0)
     assert bits.tolist() == [0x3F80, 0x3F80, 0x3F82, 0xC020]
+
+
+ROWS_SHAPES = [
+    # B, Hq, Hkv, Nq, Nk, d: GQA groups, Nq < Nk, Nq > Nk (empty causal rows)
+    (2, 6, 3, 23, 23, 8),
+    (3, 4, 1, 11, 29, 4),
+    (2, 4, 2, 31, 9, 16),
+]
+
+
+@pytest.mark.parametrize("shape", ROWS_SHAPES)
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_variant_equals_full_definition(shape, causal):
+    """oracle.attn_fwd_rows decodes a flat row index r = (b*Hq + h)*Nq + i on its
+    own; the sampled full-size checks rest on it.  Every selected row must be
+    the same bits as that row of the (pinned) full definition, and a decode
+    that swaps b/h/i or uses a wrong output stride fails here: the rows are
+    scattered over every batch, head and position, in shuffled order, with
+    repeats."""
+    B, Hq, Hkv, Nq, Nk, d = shape
+    q, k, v = rand_qkv(*shape, seed=29)
+    scale = 0.37
+    o, lse = oracle.attn_fwd(q, k, v, causal, scale)
+    rng = np.random.default_rng(5)
+    total = B * Hq * Nq
+    rows = np.concatenate([rng.permutation(total), rng.integers(0, total, size=17)])
+    ro, rl = oracle.attn_fwd_rows(q, k, v, causal, scale, rows)
+    b, h, i = rows // (Hq * Nq), (rows // Nq) % Hq, rows % Nq
+    assert np.array_equal(ro, o[b, i, h, :])
+    assert np.array_equal(rl, lse[b, h, i])
+    if causal and Nq > Nk:
+        assert np.isneginf(rl).any()  # the empty rows are among those checked
