@@ -233,6 +233,15 @@ int encode_rows(CUtensorMap* m, const void* ptr, int rows, int cols, int box_row
   return encode_cached(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides, box);
 }
 
+// The same matrix as a rank-2 map (cols, rows), for the 2-D tiled loads and
+// stores of the A@B+C epilogue.
+int encode_rows_2d(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows) {
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  return encode_cached(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box);
+}
+
 // Rows that see no key (Nk == 0): O = 0 and LSE = -inf for batches
 // [b0, b0 + nb) and query heads [h0, h0 + nh) of the [B, Nq, Hq, d] output.
 __global__ void empty_rows_kernel(__nv_bfloat16* o, float* lse, int Nq, int Hq, int d, int b0, int nb, int h0,
@@ -313,6 +322,7 @@ bool fill_params(FwdParams* p, void* o, float* lse, int B, int Hq, int Hkv, int 
   // K/V tiles through L2
   const long long kv_bytes = 2ll * part.nb * Nk * (part.nh / p->group) * Cfg::D * Cfg::ELEM;
   p->qb_major = (Cfg::CAUSAL && kv_bytes <= (48ll << 20)) ? 1 : 0;
+  p->band = 0;
   p->sl2 = scale * 1.4426950408889634f;
   p->dq = dq;
   p->dk = dk;
@@ -365,7 +375,19 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((rc = encode_qkv<Cfg>(&tq, &tk, &tv, q, k, v, B, Hq, Hkv, Nq, Nk)) != ATTN_OK) return rc;
   FwdParams p;
   if (!fill_params<Cfg>(&p, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, part)) return ATTN_ERR_UNSUPPORTED;
-  const dim3 grid((unsigned)p.n_qblocks, (unsigned)part.nh, (unsigned)part.nb);
+  dim3 grid((unsigned)p.n_qblocks, (unsigned)part.nh, (unsigned)part.nb);
+  if (Cfg::CAUSAL) {
+    // causal blocks differ in length: longest first within bands of (batch,
+    // head) pairs whose K and V together fit in about 48 MB of L2 (query heads
+    // of one key/value group are adjacent, so a band holds whole groups'
+    // worth of K/V); one 1-D grid
+    const long long kv_pair = 2ll * Nk * Cfg::D * Cfg::ELEM / p.group;  // K/V bytes per query head
+    long long band = (48ll << 20) / (kv_pair > 0 ? kv_pair : 1);
+    const long long nbh = (long long)part.nb * part.nh;
+    band = band < 1 ? 1 : (band > nbh ? nbh : band);
+    p.band = (int)band;
+    grid = dim3((unsigned)p.n_items, 1u, 1u);
+  }
   attn_fwd_kernel<Cfg><<<grid, Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -535,15 +557,19 @@ __global__ void set_float_kernel(float* p, float v) { *p = v; }
 // amax word, the amax pass, the quantising pass.  `amax` is one word of
 // device scratch (the caller's workspace or the library's static array).
 template <bool ROT>
-int launch_prep_passes(const CUtensorMap& tx, const CUtensorMap& tx8, const PrepParams& p, int grid, DeviceState* st,
+int launch_prep_passes(const CUtensorMap& tx, const CUtensorMap& tx8, const PrepParams& p, DeviceState* st,
                        cudaStream_t s) {
   static std::atomic<unsigned> attr_a[kMaxDevices], attr_q[kMaxDevices];
   int rc;
   if ((rc = set_smem_once(fp8_prep_kernel<ROT, false>, (int)PrepCfg<false>::SMEM_BYTES, attr_a, st)) != ATTN_OK ||
       (rc = set_smem_once(fp8_prep_kernel<ROT, true>, (int)PrepCfg<true>::SMEM_BYTES, attr_q, st)) != ATTN_OK)
     return rc;
-  fp8_prep_kernel<ROT, false><<<grid, kPrepRows, PrepCfg<false>::SMEM_BYTES, s>>>(tx, tx8, p);
-  fp8_prep_kernel<ROT, true><<<grid, kPrepRows, PrepCfg<true>::SMEM_BYTES, s>>>(tx, tx8, p);
+  const int ga = p.n_tiles < PrepCfg<false>::BLOCKS_PER_SM * st->num_sms ? p.n_tiles
+                                                                        : PrepCfg<false>::BLOCKS_PER_SM * st->num_sms;
+  const int gq = p.n_tiles < PrepCfg<true>::BLOCKS_PER_SM * st->num_sms ? p.n_tiles
+                                                                       : PrepCfg<true>::BLOCKS_PER_SM * st->num_sms;
+  fp8_prep_kernel<ROT, false><<<ga, kPrepRows, PrepCfg<false>::SMEM_BYTES, s>>>(tx, tx8, p);
+  fp8_prep_kernel<ROT, true><<<gq, kPrepRows, PrepCfg<true>::SMEM_BYTES, s>>>(tx, tx8, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -577,10 +603,8 @@ int launch_prep(const void* x, void* x8, float* descale, unsigned int* amax, lon
   p.descale = descale;
   p.err = st->err;
   p.timeout_ns = timeout_ns();
-  const int grid = p.n_tiles < 2 * st->num_sms ? p.n_tiles : 2 * st->num_sms;  // two blocks per SM
   if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), s) != cudaSuccess) return ATTN_ERR_CUDA;
-  return signs != nullptr ? launch_prep_passes<true>(tx, tx8, p, grid, st, s)
-                          : launch_prep_passes<false>(tx, tx8, p, grid, st, s);
+  return signs != nullptr ? launch_prep_passes<true>(tx, tx8, p, st, s) : launch_prep_passes<false>(tx, tx8, p, st, s);
 }
 
 int fill_empty(void* o, float* lse, int B, int Hq, int Nq, int d, const Part& pt, cudaStream_t s) {
@@ -830,14 +854,19 @@ int attn_gemm_add(const void* a, const void* b, const void* c, void* d, int M, i
   if (rc != ATTN_OK) return rc;
   static std::atomic<unsigned> attr_set[kMaxDevices];
   if ((rc = set_smem_once(gemm_add_kernel, (int)GemmCfg::SMEM_BYTES, attr_set, st)) != ATTN_OK) return rc;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc, td;
   std::memset(&ta, 0, sizeof(ta));
   std::memset(&tb, 0, sizeof(tb));
+  std::memset(&tc, 0, sizeof(tc));
   if (K > 0 && (encode_rows(&ta, a, M, K, GemmCfg::BM) != ATTN_OK || encode_rows(&tb, b, K, N, GemmCfg::BK) != ATTN_OK))
     return ATTN_ERR_CUDA;
+  // C and D move by 2-D tiled TMA (the kernel's loads and stores of them are
+  // .2d operations): rank-2 maps, boxes of 64 columns x 128 rows
+  if ((c != nullptr && encode_rows_2d(&tc, c, M, N, GemmCfg::BM) != ATTN_OK) ||
+      encode_rows_2d(&td, d, M, N, GemmCfg::BM) != ATTN_OK)
+    return ATTN_ERR_CUDA;
   GemmParams p;
-  p.c = static_cast<const __nv_bfloat16*>(c);
-  p.d = static_cast<__nv_bfloat16*>(d);
+  p.has_c = c != nullptr ? 1 : 0;
   p.M = M;
   p.N = N;
   p.K = K;
@@ -850,7 +879,7 @@ int attn_gemm_add(const void* a, const void* b, const void* c, void* d, int M, i
   p.timeout_ns = timeout_ns();
   const int nblk = p.n_tiles < st->num_sms ? p.n_tiles : st->num_sms;
   gemm_add_kernel<<<dim3((unsigned)nblk), GemmCfg::NTHREADS, GemmCfg::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
-      ta, tb, p);
+      ta, tb, tc, td, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

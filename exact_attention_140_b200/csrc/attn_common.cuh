@@ -21,6 +21,11 @@ struct FwdParams {
   int n_qblocks;    // ceil(Nq / (128 * NQT))
   int n_items;      // nb * nh * n_qblocks work items
   int qb_major;     // 1: order items by query block (longest first) across heads; 0: head-major
+  // one-block-per-item kernel: band > 0 runs a 1-D grid in which the
+  // (batch, head) pairs are cut into bands of `band` pairs, bands one after
+  // another, and within a band the items go longest query block first across
+  // its pairs; 0: grid (query block, head, batch x window)
+  int band;
   float sl2;        // scale * log2(e)
   // split-KV (one-block-per-item kernel): the keys are cut into n_splits
   // windows of kv_chunk keys (a multiple of the key tile); window s of batch b

@@ -78,11 +78,28 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
   const WaitCtx wc{abort_flag, p.err, p.timeout_ns};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qb = p.n_qblocks - 1 - (int)blockIdx.x;  // longest causal blocks first
   const int g = Cfg::PACK ? p.pack : 1;  // query heads stacked per tile row group
-  // query head, or key/value head when packed (grid y covers the launch's heads)
-  const int hy = (g > 1 ? p.h0 / g : p.h0) + (int)blockIdx.y;
-  const int b = p.b0 + (int)blockIdx.z / p.n_splits, split = (int)blockIdx.z % p.n_splits;
+  int qb, hy, b, split;
+  if (p.band > 0) {
+    // longest-first within bands of (batch, head) pairs: a band's K/V stay in
+    // L2 while its blocks run, and the hardware hands out blocks in this
+    // order as SMs free up, so the long causal blocks do not end up last
+    const int L = (int)blockIdx.x, nbh = p.nb * p.nh;
+    const int bi = L / (p.band * p.n_qblocks);
+    const int within = L - bi * p.band * p.n_qblocks;
+    const int bsz = nbh - bi * p.band < p.band ? nbh - bi * p.band : p.band;
+    const int r = bi * p.band + within % bsz;
+    qb = p.n_qblocks - 1 - within / bsz;
+    hy = p.h0 + r % p.nh;
+    b = p.b0 + r / p.nh;
+    split = 0;
+  } else {
+    qb = p.n_qblocks - 1 - (int)blockIdx.x;  // longest causal blocks first
+    // query head, or key/value head when packed (grid y covers the launch's heads)
+    hy = (g > 1 ? p.h0 / g : p.h0) + (int)blockIdx.y;
+    b = p.b0 + (int)blockIdx.z / p.n_splits;
+    split = (int)blockIdx.z % p.n_splits;
+  }
   // key window of this block: [kv0, kv0 + nk), `shift` keys after it
   const int kv0 = split * p.kv_chunk;
   const int nk = p.Nk - kv0 < p.kv_chunk ? p.Nk - kv0 : p.kv_chunk;

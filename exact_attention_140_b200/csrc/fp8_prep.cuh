@@ -12,8 +12,10 @@
 //   * thread t of a 128-thread block owns row t of the tile: it reads the row
 //     from shared memory (the swizzle spreads the 16-byte chunks of eight
 //     consecutive rows over all banks, so the reads are conflict-free), and
-//     runs the whole fast Walsh-Hadamard transform in registers (level 0 in
-//     scalar fp32, levels 1-6 as packed fp32x2 butterflies) -- no shuffles;
+//     runs the whole fast Walsh-Hadamard transform in registers -- no
+//     shuffles: a packed fp32x2 register holds elements k and k + 64, so six
+//     of the seven butterfly levels are packed operations and only the last
+//     one is scalar (the amax pass needs only |a| + |b| of it);
 //   * the random signs are applied as XOR masks on the bf16 sign bits before
 //     the values are widened (an exact multiplication by +-1), and 1/sqrt(d)
 //     is folded into the final scale: fl(max|y| * c) = max fl(|y| * c) for
@@ -43,7 +45,11 @@ constexpr float kPrepInvSqrtD = 0.08838834764831845f;        // 1/sqrt(128)
 
 template <bool QUANT>
 struct PrepCfg {
-  static constexpr int STAGES = QUANT ? 2 : 3;
+  // the amax pass keeps 128 values and little else per thread (under 170
+  // registers): three blocks per SM; the quantising pass needs more registers
+  // and an output buffer: two blocks per SM
+  static constexpr int BLOCKS_PER_SM = QUANT ? 2 : 3;
+  static constexpr int STAGES = 2;
   static constexpr uint32_t OFF_IN = 0;
   static constexpr uint32_t OFF_OUT = STAGES * kPrepTileBytes;
   static constexpr uint32_t OFF_BAR = OFF_OUT + (QUANT ? kPrepOutBytes : 0);
@@ -53,7 +59,7 @@ struct PrepCfg {
   static constexpr uint32_t OFF_RED = OFF_ABORT + 16;
   static constexpr uint32_t SMEM_BYTES = OFF_RED + 4 * 4 + 1024;  // + alignment slack
   static_assert(OFF_MASK % 16 == 0 && OFF_IN % 1024 == 0 && OFF_OUT % 1024 == 0, "vector and TMA alignment");
-  static_assert(2 * SMEM_BYTES <= 227 * 1024, "two blocks per SM");
+  static_assert(BLOCKS_PER_SM * (SMEM_BYTES + 1024) <= 228 * 1024, "blocks per SM");
 };
 
 struct PrepParams {
@@ -66,55 +72,66 @@ struct PrepParams {
   unsigned long long timeout_ns;
 };
 
-// Row t of the tile in stage memory `tile` (two swizzled 64-column boxes) ->
-// 128 fp32 values, signs applied (XOR masks on the bf16 sign bits), then the
-// unnormalised Walsh-Hadamard transform when ROT.  v[2k], v[2k+1] live in
-// one packed register pair P[k].
+// Row r of the tile in stage memory `tile` (two swizzled 64-column boxes) ->
+// 128 fp32 values, signs applied (XOR masks on the bf16 sign bits), then, when
+// ROT, levels 0..5 of the unnormalised Walsh-Hadamard transform.  The packed
+// register pair P[k] holds elements k and k + 64 (column k of each box), so
+// the butterflies of spans 1..32 are packed fp32x2 operations on both halves
+// at once; the last level (span 64) pairs the two halves of each P[k]:
+// y[k] = a + b, y[k + 64] = a - b for P[k] = (a, b), and is left to the
+// caller (the amax pass needs only max(|a + b|, |a - b|) = |a| + |b|).
 template <bool ROT>
 __device__ __forceinline__ void prep_load_transform(const uint8_t* tile, const uint4* mask4, int r,
                                                     uint64_t (&P)[64]) {
 #pragma unroll
-  for (int h = 0; h < 2; ++h)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint4 w = *reinterpret_cast<const uint4*>(tile + h * kPrepHalfBytes + r * 128 + ((c ^ (r & 7)) << 4));
-      if constexpr (ROT) {
-        const uint4 m = mask4[h * 8 + c];
-        w.x ^= m.x;
-        w.y ^= m.y;
-        w.z ^= m.z;
-        w.w ^= m.w;
-      }
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xFFFF0000u);
-        if constexpr (ROT) {
-          // level 0 of the transform (span 1) on the pair as it is widened
-          P[h * 32 + c * 4 + e] = ptx::f2(lo + hi, lo - hi);
-        } else {
-          P[h * 32 + c * 4 + e] = ptx::f2(lo, hi);
-        }
-      }
+  for (int c = 0; c < 8; ++c) {
+    const int off = r * 128 + ((c ^ (r & 7)) << 4);
+    uint4 w0 = *reinterpret_cast<const uint4*>(tile + off);                   // elements 8c .. 8c+7
+    uint4 w1 = *reinterpret_cast<const uint4*>(tile + kPrepHalfBytes + off);  // elements 64+8c ..
+    if constexpr (ROT) {
+      const uint4 m0 = mask4[c], m1 = mask4[8 + c];
+      w0.x ^= m0.x;
+      w0.y ^= m0.y;
+      w0.z ^= m0.z;
+      w0.w ^= m0.w;
+      w1.x ^= m1.x;
+      w1.y ^= m1.y;
+      w1.z ^= m1.z;
+      w1.w ^= m1.w;
     }
+    const uint32_t a[4] = {w0.x, w0.y, w0.z, w0.w}, b[4] = {w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      P[8 * c + 2 * e] = ptx::f2(__uint_as_float(a[e] << 16), __uint_as_float(b[e] << 16));
+      P[8 * c + 2 * e + 1] = ptx::f2(__uint_as_float(a[e] & 0xFFFF0000u), __uint_as_float(b[e] & 0xFFFF0000u));
+    }
+  }
   if constexpr (ROT) {
-    // levels 1..6 (spans 2..64 elements = 1..32 pairs): packed butterflies
 #pragma unroll
     for (int sp = 1; sp < 64; sp <<= 1)
 #pragma unroll
       for (int k = 0; k < 64; ++k)
         if ((k & sp) == 0) {
-          const uint64_t a = P[k], b = P[k + sp];
-          P[k] = ptx::fadd2(a, b);
-          P[k + sp] = ptx::fsub2(a, b);
+          const uint64_t x = P[k], y = P[k + sp];
+          P[k] = ptx::fadd2(x, y);
+          P[k + sp] = ptx::fsub2(x, y);
         }
   }
+}
+
+// Element j (0..127) of the transformed row: the last butterfly level when ROT.
+template <bool ROT>
+__device__ __forceinline__ float prep_elem(const uint64_t (&P)[64], int j) {
+  float a, b;
+  ptx::unf2(P[j & 63], a, b);
+  if constexpr (ROT) return j < 64 ? a + b : a - b;
+  return j < 64 ? a : b;
 }
 
 // One pass over the tensor: QUANT = false accumulates amax (one atomicMax per
 // block), QUANT = true writes the codes and, from block 0, the descale.
 template <bool ROT, bool QUANT>
-__global__ void __launch_bounds__(kPrepRows, 2)
+__global__ void __launch_bounds__(kPrepRows, PrepCfg<QUANT>::BLOCKS_PER_SM)
     fp8_prep_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmX8,
                     const PrepParams p) {
   using C = PrepCfg<QUANT>;
@@ -194,8 +211,12 @@ __global__ void __launch_bounds__(kPrepRows, 2)
       for (int i = 0; i < 64; ++i) {
         float a, b;
         ptx::unf2(P[i], a, b);
-        m0 = fmaxf(m0, fabsf(a));
-        m1 = fmaxf(m1, fabsf(b));
+        if constexpr (ROT) {
+          m0 = fmaxf(m0, fabsf(a) + fabsf(b));  // = max(|a + b|, |a - b|), also in fp32
+        } else {
+          m0 = fmaxf(m0, fabsf(a));
+          m1 = fmaxf(m1, fabsf(b));
+        }
       }
     } else {
       uint8_t* out = sgen + C::OFF_OUT;
@@ -204,10 +225,9 @@ __global__ void __launch_bounds__(kPrepRows, 2)
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          float a, b, cc, d;
-          ptx::unf2(P[c * 8 + 2 * e], a, b);
-          ptx::unf2(P[c * 8 + 2 * e + 1], cc, d);
-          w[e] = ptx::pack_e4m3x4(a * mult, b * mult, cc * mult, d * mult);
+          const int j = 16 * c + 4 * e;
+          w[e] = ptx::pack_e4m3x4(prep_elem<ROT>(P, j) * mult, prep_elem<ROT>(P, j + 1) * mult,
+                                  prep_elem<ROT>(P, j + 2) * mult, prep_elem<ROT>(P, j + 3) * mult);
         }
         *reinterpret_cast<uint4*>(out + tid * 128 + ((c ^ (tid & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }

@@ -12,15 +12,24 @@
 //   warps 0..7   epilogue, two warpgroups: warpgroup g takes columns
 //                [128 g, 128 g + 128) of the tile, warp w its TMEM lanes
 //                32 (w % 4) .. +31 (one tile row per thread); it reads the
-//                accumulator from TMEM, adds C and stores D (bf16);
-//   warp 8       TMA producer: A (K-major) and B (MN-major) tiles of BK = 64
-//                through a STAGES-deep shared-memory ring;
+//                accumulator from TMEM, adds C from shared memory, writes D
+//                back over C in shared memory, and one thread stores the
+//                tile with TMA;
+//   warp 8       TMA producer: A (K-major) and B (MN-major) blocks of BK = 64
+//                through a STAGES-deep ring, and each tile's C into one of two
+//                tile buffers;
 //   warp 9       MMA issuer (converged warp, elected lane), also allocates
 //                tensor memory: tile i accumulates into TMEM columns
 //                [256 (i % 2), +256), so the products of tile i + 1 run while
 //                the epilogue drains tile i.
+// C and D move as whole 128-byte-swizzled boxes (64 columns x 128 rows) by
+// TMA, so HBM sees full lines in both directions; a thread reads and writes
+// the 16-byte chunks of its own row, which the swizzle spreads over all banks.
+// Tile buffer b is reused by tile i + 2 once the TMA store of tile i has read
+// it (barrier cd_free).
 // Layouts: A [M, K], B [K, N], C and D [M, N], row-major bf16; fp32
-// accumulation; D = bf16(A B + C) with round-to-nearest-even.
+// accumulation; D = bf16(A B + C) with round-to-nearest-even.  C may be D
+// itself: a tile's C is loaded before its D is stored, and tiles are disjoint.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -33,26 +42,30 @@ namespace attn {
 
 struct GemmCfg {
   static constexpr int BM = 128, BN = 256, BK = 64;
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = 2;
   static constexpr uint32_t A_BYTES = BM * 128;            // 128 rows of 64 bf16
   static constexpr uint32_t B_CHUNK = BK * 128;            // 64 K-rows of 64 N-columns
   static constexpr uint32_t B_BYTES = B_CHUNK * (BN / 64);
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t BOX_BYTES = BM * 128;          // 128 rows of 64 bf16 (one C/D box)
+  static constexpr uint32_t CD_BYTES = BOX_BYTES * (BN / 64);
   static constexpr int B_FULL = 0, B_EMPTY = STAGES, B_ACCF = 2 * STAGES, B_ACCE = 2 * STAGES + 2;
-  static constexpr int B_DRAIN = 2 * STAGES + 4, NBAR = 2 * STAGES + 5;
-  static constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr int B_CFULL = 2 * STAGES + 4, B_CDFREE = 2 * STAGES + 6;
+  static constexpr int B_DRAIN = 2 * STAGES + 8, NBAR = 2 * STAGES + 9;
+  static constexpr uint32_t OFF_CD = STAGES * STAGE_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_CD + 2 * CD_BYTES;
   static constexpr uint32_t OFF_SLOT = OFF_BAR + NBAR * 8;
   static constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
   static constexpr uint32_t SMEM_BYTES = OFF_ABORT + 4 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per block");
+  static_assert(OFF_CD % 1024 == 0 && CD_BYTES % 1024 == 0, "swizzled boxes need 1024-byte alignment");
   static constexpr int EPI_WARPS = 8, TMA_WARP = 8, MMA_WARP = 9, NTHREADS = 384;
   static constexpr int EPI_THREADS = 32 * EPI_WARPS;
   static constexpr uint32_t IDESC = ptx::idesc<false>(BM, BN, true);  // B is MN-major
 };
 
 struct GemmParams {
-  const __nv_bfloat16* c;  // [M, N] or nullptr
-  __nv_bfloat16* d;        // [M, N]
+  int has_c;  // 0: D = A B
   int M, N, K;
   int tiles_m, n_tiles, k_steps;
   unsigned int* err;
@@ -61,6 +74,7 @@ struct GemmParams {
 
 __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
     gemm_add_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                     const GemmParams p) {
   using G = GemmCfg;
   extern __shared__ uint8_t smem_raw[];
@@ -84,6 +98,8 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(bar(G::B_ACCF + a), 1);
       ptx::mbar_init(bar(G::B_ACCE + a), G::EPI_THREADS);
+      ptx::mbar_init(bar(G::B_CFULL + a), 1);
+      ptx::mbar_init(bar(G::B_CDFREE + a), 1);
     }
     ptx::mbar_init(bar(G::B_DRAIN), 1);
     *abort_flag = 0u;
@@ -92,6 +108,8 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
   if (warp == G::TMA_WARP && lane == 0) {
     ptx::prefetch_tmap(&tmA);
     ptx::prefetch_tmap(&tmB);
+    if (p.has_c) ptx::prefetch_tmap(&tmC);
+    ptx::prefetch_tmap(&tmD);
   }
   if (warp == G::MMA_WARP) {
     ptx::tmem_alloc(sbase + G::OFF_SLOT, 512);
@@ -106,69 +124,71 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int wg = warp >> 2, wq = warp & 3;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const int r = wq * 32 + lane;  // this thread's row of the tile
     bool ok = true;
+    int stored = 0;  // TMA store groups committed by thread 0
     for (int k = 0; ok; ++k) {
       const int tile = tile_at(k);
       if (tile < 0) break;
-      const int acc = k & 1;
+      const int acc = k & 1, buf = k & 1;
       const int m0 = (tile % p.tiles_m) * G::BM, n0 = (tile / p.tiles_m) * G::BN;
-      const int row = m0 + wq * 32 + lane;
-      const bool row_ok = row < p.M;
-      const long long row_off = (long long)row * p.N;
-      // C does not depend on the products: this thread's 128 values of it are
-      // requested before the accumulator is waited for, so the loads overlap
-      // the wait and each other (N is a multiple of 8: 8-column groups are whole).
-      // Plain (coherent) loads: C may be D itself (an in-place update), and the
-      // thread that reads an element of C is the one that later writes it to D.
-      uint4 cr[4][4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int col = n0 + wg * 128 + 32 * c + 8 * g;
-          cr[c][g] = (p.c != nullptr && row_ok && col < p.N)
-                         ? *reinterpret_cast<const uint4*>(p.c + row_off + col)
-                         : make_uint4(0u, 0u, 0u, 0u);
-        }
       ok = wait_bar<kRoleSoftmax>(bar(G::B_ACCF + acc), (uint32_t)((k >> 1) & 1), wc, kSiteODone);
-      ok = __all_sync(0xffffffffu, ok);
+      if (ok && p.has_c)  // this tile's C is in the buffer
+        ok = wait_bar<kRoleSoftmax>(bar(G::B_CFULL + buf), (uint32_t)((k >> 1) & 1), wc, kSiteVFull);
+      else if (ok && k >= 2)  // no C: the store of tile k - 2 must have read the buffer
+        ok = wait_bar<kRoleSoftmax>(bar(G::B_CDFREE + buf), (uint32_t)(((k >> 1) - 1) & 1), wc, kSiteVEmpty);
+      // all epilogue warps take the same branch (they meet at a named barrier below)
+      ok = ptx::bar_red_and(1, G::EPI_THREADS, ok);
       if (!ok) break;
       ptx::tc_fence_after();
+      uint8_t* cd = sgen + G::OFF_CD + (uint32_t)buf * G::CD_BYTES;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const int col0 = n0 + wg * 128 + 32 * c;
-        uint32_t r[32];
+        uint32_t rr[32];
         if (p.k_steps > 0) {
-          ptx::tmem_ld32(tmem + lane_off + (uint32_t)(acc * 256 + wg * 128 + 32 * c), r);
-          ptx::tmem_wait_ld_dep(r);
+          ptx::tmem_ld32(tmem + lane_off + (uint32_t)(acc * 256 + wg * 128 + 32 * c), rr);
+          ptx::tmem_wait_ld_dep(rr);
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = 0u;
+          for (int e = 0; e < 32; ++e) rr[e] = 0u;
         }
-        if (row_ok) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int col = col0 + 8 * g;
-            if (col < p.N) {
-              const uint32_t w4[4] = {cr[c][g].x, cr[c][g].y, cr[c][g].z, cr[c][g].w};
-              uint32_t w[4];
+        for (int g = 0; g < 4; ++g) {
+          // columns wg*128 + 32c + 8g .. +7: box 2wg + c/2, chunk 4(c%2) + g of row r
+          const int box = 2 * wg + c / 2, q = 4 * (c % 2) + g;
+          uint4* chunk = reinterpret_cast<uint4*>(cd + box * G::BOX_BYTES + r * 128 + ((q ^ (r & 7)) << 4));
+          const uint4 cv = p.has_c ? *chunk : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t w4[4] = {cv.x, cv.y, cv.z, cv.w};
+          uint32_t w[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                w[e] = ptx::pack_bf16x2(__uint_as_float(r[8 * g + 2 * e]) + __uint_as_float(w4[e] << 16),
-                                        __uint_as_float(r[8 * g + 2 * e + 1]) + __uint_as_float(w4[e] & 0xFFFF0000u));
-              *reinterpret_cast<uint4*>(p.d + row_off + col) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-          }
+          for (int e = 0; e < 4; ++e)
+            w[e] = ptx::pack_bf16x2(__uint_as_float(rr[8 * g + 2 * e]) + __uint_as_float(w4[e] << 16),
+                                    __uint_as_float(rr[8 * g + 2 * e + 1]) + __uint_as_float(w4[e] & 0xFFFF0000u));
+          *chunk = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      // this accumulator has been read out: tile k + 2 may overwrite it
+      // the accumulator has been read out: tile k + 2 may overwrite it
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar(G::B_ACCE + acc));
+      // D is in the buffer: every epilogue thread's writes reach the async
+      // proxy, then one thread stores the four boxes
+      ptx::fence_proxy_async_smem();
+      asm volatile("bar.sync 1, %0;" ::"n"(G::EPI_THREADS) : "memory");
+      if (threadIdx.x == 0) {
+        const uint32_t cds = sbase + G::OFF_CD + (uint32_t)buf * G::CD_BYTES;
+#pragma unroll
+        for (int j = 0; j < G::BN / 64; ++j) ptx::tma_store_2d(&tmD, cds + (uint32_t)j * G::BOX_BYTES, n0 + 64 * j, m0);
+        ptx::bulk_commit();
+        ++stored;
+        ptx::bulk_wait_read0();  // the stores have read the buffer
+        ptx::mbar_arrive(bar(G::B_CDFREE + buf));
+      }
     }
+    if (threadIdx.x == 0 && stored > 0) ptx::bulk_wait0();  // D is written before the block exits
   } else if (warp == G::TMA_WARP) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int issued[G::STAGES];
+      int issued[G::STAGES], c_issued[2] = {0, 0};
 #pragma unroll
       for (int s = 0; s < G::STAGES; ++s) issued[s] = 0;
       int it = 0;  // k-blocks issued into the ring, across tiles
@@ -194,12 +214,31 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
             ptx::tma_load_4d(st + G::A_BYTES + (uint32_t)c * G::B_CHUNK, &tmB, fb, n0 + 64 * c, kb * G::BK, 0, 0);
           ++issued[s];
         }
+        if (!ok) break;
+        if (p.has_c) {
+          // C of tile k into buffer k % 2, once the store of tile k - 2 has read it
+          const int buf = k & 1;
+          if (k >= 2 && !wait_bar<kRoleProducer>(bar(G::B_CDFREE + buf), (uint32_t)(((k >> 1) - 1) & 1), wc,
+                                                  kSiteVEmpty))
+            break;
+          const uint32_t fb = bar(G::B_CFULL + buf);
+          const uint32_t cds = sbase + G::OFF_CD + (uint32_t)buf * G::CD_BYTES;
+          ptx::mbar_arrive_expect_tx(fb, G::CD_BYTES);
+#pragma unroll
+          for (int j = 0; j < G::BN / 64; ++j)
+            ptx::tma_load_2d(cds + (uint32_t)j * G::BOX_BYTES, &tmC, fb, n0 + 64 * j, m0);
+          ++c_issued[buf];
+        }
       }
       // every issued copy must land before the block may exit
 #pragma unroll
       for (int s = 0; s < G::STAGES; ++s)
         if (issued[s] > 0)
           wait_bar_drain<kRoleProducer>(bar(G::B_FULL + s), (uint32_t)((issued[s] - 1) & 1), wc, kSiteKFull);
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+        if (c_issued[b] > 0)
+          wait_bar_drain<kRoleProducer>(bar(G::B_CFULL + b), (uint32_t)((c_issued[b] - 1) & 1), wc, kSiteVFull);
     }
   } else if (warp == G::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
