@@ -518,7 +518,7 @@ constexpr int kPersistentMaxNk = 1024;
 //   in columns of its own (S 128 + P 64 + O 64 = 256 columns per stream).
 template <bool C> using CfgD64 = FwdCfg<64, 128, 2, 3, 3, C, false, 3>;
 template <bool C> using CfgD64Short = FwdCfg<64, 128, 1, 3, 3, C, false, 2, 1, true, 2>;
-template <bool C> using CfgD128 = FwdCfg<128, 128, 2, 2, 2, C, false, 2>;
+template <bool C> using CfgD128 = FwdCfg<128, 128, 2, 2, 2, C, false, C ? 2 : 1>;
 template <bool C> using CfgD128Short = FwdCfg<128, 128, 2, 2, 2, C, false, 0>;
 template <bool C> using CfgD256 = FwdCfg<256, 64, 1, 2, 2, C, false, 0>;
 template <bool C> using CfgFP8 = FwdCfg<128, 128, 2, 3, 3, C, true, 3>;

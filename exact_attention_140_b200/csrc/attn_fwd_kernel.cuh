@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
     for (int i = 0; i < NQT * SB; ++i) {
       ptx::mbar_init(bar(Cfg::B_SFULL + i), 1);
       ptx::mbar_init(bar(Cfg::B_PFULL + i), 128);
+      ptx::mbar_init(bar(Cfg::B_PHALF + i), 128);
     }
     for (int t = 0; t < NQT; ++t) {
       ptx::mbar_init(bar(Cfg::B_ODONE + t), 1);
@@ -224,6 +225,10 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         l *= alpha;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      const bool resc_any = __any_sync(0xffffffffu, resc);
+      // P released in two halves (non-causal: measured faster; with causal
+      // masks the extra live state costs more than the overlap gains)
+      constexpr bool kHalfP = !Cfg::CAUSAL;
       // ---- exponentiate 32 columns at a time; each chunk's packed P is
       // stored at once (over score columns already read), so the registers of
       // a chunk die before the next chunk is processed
@@ -275,6 +280,15 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
             ptx::tmem_st8(s_taddr + (uint32_t)(PW * ch), pk);
           else
             ptx::tmem_st16(s_taddr + (uint32_t)(PW * ch), pk);
+          if (kHalfP && ch == BN / 64 - 1 && !resc_any) {
+            // the first half of P is in tensor memory: the P V over the first
+            // half of the keys can start while the second half is
+            // exponentiated (a warp that must rescale O first releases it
+            // after the rescale instead)
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar(Cfg::B_PHALF + si));
+          }
         }
       };
       if (partial)
@@ -287,7 +301,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         l += la + lb;
       }
       ptx::tmem_wait_st();
-      if (__any_sync(0xffffffffu, resc)) {
+      if (resc_any) {
         // O_t must hold exactly the products of key tiles < j: wait for
         // PV(t, j-1).  Whenever S(t, j) is ready, PV(t, j-2) has completed (it
         // was issued before QK(t, j)) and PV(t, j) is not issued yet, so the
@@ -310,6 +324,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         ptx::tmem_wait_st();
       }
       ptx::tc_fence_before();
+      if (!Cfg::CAUSAL && resc_any) ptx::mbar_arrive(bar(Cfg::B_PHALF + si));
       ptx::mbar_arrive(bar(Cfg::B_PFULL + si));
     }
     // ------------------------------------------------------------ epilogue
@@ -462,15 +477,23 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       };
       auto issue_pv = [&](int t, int jj) -> bool {
         const int si = t * SB + jj % SB;
-        if (!wait_bar_warp<kRoleMma>(bar(Cfg::B_PFULL + si), (uint32_t)((jj / SB) & 1), wc, kSitePFull)) return false;
-        ptx::tc_fence_after();
+        const uint32_t ph = (uint32_t)((jj / SB) & 1);
         const uint32_t d_t = tmem + (uint32_t)(Cfg::O_COL0 + t * D);
         const uint32_t a_t = tmem + (uint32_t)(si * BN);
         const uint64_t bd0 = ptx::sdesc_sw128(v_s + (jj % VST) * Cfg::KV_BYTES, Cfg::CH_KV, 1024u);
+        // non-causal: the first half of the keys as soon as their P is
+        // written, the rest when the whole P is; causal: all at once
 #pragma unroll
-        for (int kk = 0; kk < Cfg::PV_STEPS; ++kk) {
-          const uint64_t bd = bd0 + (uint64_t)(((uint32_t)kk * Cfg::KSTEP * 128u) >> 4);
-          ptx::warp_mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+        for (int half = Cfg::CAUSAL ? 1 : 0; half < 2; ++half) {
+          if (!wait_bar_warp<kRoleMma>(bar((half == 0 ? Cfg::B_PHALF : Cfg::B_PFULL) + si), ph, wc, kSitePFull))
+            return false;
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int kk = (Cfg::CAUSAL ? 0 : half * Cfg::PV_STEPS / 2); kk < (half + 1) * Cfg::PV_STEPS / 2; ++kk) {
+            const uint64_t bd = bd0 + (uint64_t)(((uint32_t)kk * Cfg::KSTEP * 128u) >> 4);
+            ptx::warp_mma_ts<Cfg::FP8>(d_t, a_t + (uint32_t)kk * 8u, bd, Cfg::IDESC_PV,
+                                       (jj > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         ptx::warp_commit(bar(Cfg::B_ODONE + t));
         if (jj == n_kv[t] - 1) ptx::warp_commit(bar(Cfg::B_OFINAL + t));
