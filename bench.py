@@ -401,7 +401,7 @@ def run_ours(args, cfg, name):
     else:
         roofline = tensor_roofline(achieved, peaks, float(np.sum(kern_ms)) * 1e-3, fp8)
         roofline.update(traffic=traffic,
-                        kernel="attn_fwd_persistent_kernel" if ea.attn_fwd_schedule(N) == 1 else "attn_fwd_kernel")
+                        kernel="attn_fwd_persistent_kernel" if ea.attn_fwd_schedule(N, d, causal) == 1 else "attn_fwd_kernel")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,

@@ -69,7 +69,7 @@ _lib.attn_kv_tile_count.argtypes = [_I] * 6
 _lib.attn_kv_tile_count.restype = _I
 _lib.attn_tile_kind.argtypes = [_I] * 7
 _lib.attn_tile_kind.restype = _I
-_lib.attn_fwd_schedule.argtypes = [_I]
+_lib.attn_fwd_schedule.argtypes = [_I] * 3
 _lib.attn_fwd_schedule.restype = _I
 _lib.attn_debug_unsatisfied_wait.argtypes = [_LL, _vp]
 _lib.attn_debug_unsatisfied_wait.restype = _I
@@ -232,9 +232,9 @@ def attn_tile_kind_window(row0, row1, kt, Nq, Nk, shift, bn, causal) -> int:
     return int(_lib.attn_tile_kind_window(row0, row1, kt, Nq, Nk, shift, bn, int(causal)))
 
 
-def attn_fwd_schedule(Nk) -> int:
-    """1 if attn_fwd runs the persistent kernel for Nk keys, 0 for one block per item."""
-    return int(_lib.attn_fwd_schedule(Nk))
+def attn_fwd_schedule(Nk, d, causal) -> int:
+    """1 if attn_fwd runs the persistent kernel for Nk keys at head size d, 0 for one block per item."""
+    return int(_lib.attn_fwd_schedule(Nk, d, int(causal)))
 
 
 def attn_debug_unsatisfied_wait(limit_ns: int, stream=None, raise_on_error=True):

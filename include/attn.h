@@ -284,14 +284,16 @@ int attn_tile_kind_window(int row0, int row1, int kt, int Nq, int Nk, int shift,
 int attn_gemm_add(const void *a, const void *b, const void *c, void *d, int M, int N, int K, void *stream);
 
 /*
- * Which kernel attn_fwd / attn_fwd_fp8 launch for a key range of Nk keys:
- * 1 = the persistent kernel (one block per SM looping over the work items;
- * used for short key ranges, whose items are short), 0 = one block per work
- * item.  Both compute the same result.  Host-only; -1 if Nk < 0.  The page
- * set describes one block per (batch, head, query block); the persistent
- * schedule is this library's own.
+ * Which kernel attn_fwd / attn_fwd_fp8 launch for a key range of Nk keys at
+ * head size d (64, 128, 256) with the causal flag: 1 = the persistent kernel
+ * (one block per SM looping over the work items; used for short key ranges,
+ * Nk <= 1024, whose items are short), 0 = one block per work item (longer
+ * ranges, and causal launches at d = 128, where the blocks of uneven causal
+ * items are handed out longest first).  Both compute the same result.
+ * Host-only; -1 for invalid arguments.  The page set describes one block per
+ * (batch, head, query block); the persistent schedule is this library's own.
  */
-int attn_fwd_schedule(int Nk);
+int attn_fwd_schedule(int Nk, int d, int causal);
 
 /*
  * Debug hook for the failure path: launches one block that waits, with the

@@ -94,8 +94,13 @@ def test_error_raises():
 
 def test_schedule_boundary():
     # persistent kernel for key ranges up to 1024, one block per item above
-    assert ea.attn_fwd_schedule(-1) == -1
-    assert [ea.attn_fwd_schedule(n) for n in (0, 1, 1024, 1025, 8192)] == [1, 1, 1, 0, 0]
+    assert ea.attn_fwd_schedule(-1, 128, 0) == -1
+    assert ea.attn_fwd_schedule(64, 96, 0) == -1
+    for d in (64, 128, 256):
+        assert [ea.attn_fwd_schedule(n, d, 0) for n in (0, 1, 1024, 1025, 8192)] == [1, 1, 1, 0, 0]
+    # causal: persistent up to 1024 keys at d = 64 and 256; never at d = 128
+    assert [ea.attn_fwd_schedule(n, 64, 1) for n in (1, 1024, 1025)] == [1, 1, 0]
+    assert [ea.attn_fwd_schedule(n, 128, 1) for n in (1, 1024, 1025)] == [0, 0, 0]
 
 
 def test_splitkv_argument_errors_before_any_cuda_call():
