@@ -404,9 +404,12 @@ int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, 
   if ((rc = encode_qkv<Cfg>(&tq, &tk, &tv, q, k, v, B, Hq, Hkv, Nq, Nk)) != ATTN_OK) return rc;
   FwdParams p;
   if (!fill_params<Cfg>(&p, o, lse, B, Hq, Hkv, Nq, Nk, scale, dq, dk, dv, st, part)) return ATTN_ERR_UNSUPPORTED;
+  // the output map (staged output only; otherwise an unused copy of Q's)
+  CUtensorMap to = tq;
+  if (Cfg::OST && encode_bnhd(&to, o, false, B, Nq, Hq, Cfg::D, Cfg::BM) != ATTN_OK) return ATTN_ERR_CUDA;
   const int nstreams = (p.n_items + Cfg::NS - 1) / Cfg::NS;  // blocks that find work
   const int nblk = nstreams < st->num_sms ? nstreams : st->num_sms;
-  attn_fwd_persistent_kernel<Cfg><<<dim3((unsigned)nblk), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  attn_fwd_persistent_kernel<Cfg><<<dim3((unsigned)nblk), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -525,11 +528,11 @@ bool use_persistent(int Nk, int d, bool causal) { return Nk <= kPersistentMaxNk 
 //   d = 64 short: two independent streams of one 128-row query tile each; P
 //   in columns of its own (S 128 + P 64 + O 64 = 256 columns per stream).
 template <bool C> using CfgD64 = FwdCfg<64, 128, 2, 3, 3, C, false, 3>;
-template <bool C> using CfgD64Short = FwdCfg<64, 128, 1, 3, 3, C, false, 2, 1, true, 2>;
+template <bool C> using CfgD64Short = FwdCfg<64, 128, 1, 2, 3, C, false, 2, 1, true, 2, false, true>;
 template <bool C> using CfgD128 = FwdCfg<128, 128, 2, 2, 2, C, false, C ? 2 : 1>;
 template <bool C> using CfgD128Short = FwdCfg<128, 128, 2, 2, 2, C, false, 0>;
 template <bool C> using CfgD256 = FwdCfg<256, 64, 1, 2, 2, C, false, 0>;
-template <bool C> using CfgFP8 = FwdCfg<128, 128, 2, 3, 3, C, true, 3>;
+template <bool C> using CfgFP8 = FwdCfg<128, 128, 2, 3, 3, C, true, 2>;
 
 template <template <bool> class Long, template <bool> class Short>
 int launch_sched(bool causal, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,

@@ -51,8 +51,36 @@ struct FwdParams {
 
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
 
+// Maximum of sl2 * s[c] over the visible columns c < nvis of N scores (the
+// keys of a partially masked tile form a prefix); -inf when none is visible.
+// Four independent chains of three-input max on the raw scores, one multiply
+// at the end (sl2 >= 0 keeps the order; a negative scale takes the minimum).
+template <int N>
+__device__ __forceinline__ float masked_max_scaled(const uint32_t* sr, int nvis, float sl2) {
+  if (sl2 >= 0.f) {
+    float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < N; c += 2) {
+      const float x0 = c < nvis ? __uint_as_float(sr[c]) : -INFINITY;
+      const float x1 = c + 1 < nvis ? __uint_as_float(sr[c + 1]) : -INFINITY;
+      a[(c / 2) % 4] = ptx::fmax3(a[(c / 2) % 4], x0, x1);
+    }
+    const float m = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+    return m == -INFINITY ? -INFINITY : m * sl2;
+  }
+  float a[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+#pragma unroll
+  for (int c = 0; c < N; c += 2) {
+    const float x0 = c < nvis ? __uint_as_float(sr[c]) : INFINITY;
+    const float x1 = c + 1 < nvis ? __uint_as_float(sr[c + 1]) : INFINITY;
+    a[(c / 2) % 4] = fminf(a[(c / 2) % 4], fminf(x0, x1));
+  }
+  const float m = fminf(fminf(a[0], a[1]), fminf(a[2], a[3]));
+  return m == INFINITY ? -INFINITY : m * sl2;
+}
+
 template <int D_, int BN_, int NQT_, int KST_, int VST_, bool CAUSAL_, bool FP8_, int EMU_ = 0,
-          int SB_ = (NQT_ == 1 ? 2 : 1), bool PSEP_ = false, int NS_ = 1, bool PACK_ = false>
+          int SB_ = (NQT_ == 1 ? 2 : 1), bool PSEP_ = false, int NS_ = 1, bool PACK_ = false, bool OST_ = false>
 struct FwdCfg {
   // PACK: the one-block-per-item kernel reads the head-packing factor from the
   // launch parameters (split-KV); otherwise it is compiled out
@@ -71,6 +99,11 @@ struct FwdCfg {
   static constexpr int EMU = EMU_;
   static constexpr bool CAUSAL = CAUSAL_, FP8 = FP8_;
   static constexpr int BM = 128;
+  // OST (persistent kernel, bf16): each stream stages its output tile in
+  // shared memory (the 128-byte-swizzled layout of a Q tile) and writes it
+  // with one TMA store, instead of one row per thread
+  static constexpr bool OST = OST_;
+  static_assert(!OST || (!FP8 && NQT == 1), "staged output: bf16, one query tile per stream");
   static constexpr int SB = SB_;  // score buffers per query tile
   static_assert(SB == 1 || SB == 2, "one or two score buffers");
   static constexpr int ELEM = FP8 ? 1 : 2;
@@ -114,7 +147,8 @@ struct FwdCfg {
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + NQT * QT_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr uint32_t STREAM_BYTES = OFF_V + VST * KV_BYTES;
+  static constexpr uint32_t OFF_OST = OFF_V + VST * KV_BYTES;  // output staging tile (OST)
+  static constexpr uint32_t STREAM_BYTES = OFF_OST + (OST ? (uint32_t)BM * D * 2 : 0u);
   static constexpr uint32_t OFF_BAR = NS * STREAM_BYTES;
   static constexpr uint32_t OFF_SLOT = OFF_BAR + NS * NBAR * 8;
   static constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
@@ -129,9 +163,9 @@ struct FwdCfg {
   static constexpr int TMA_WARP = SM_WARPS;
   static constexpr int MMA_WARP = SM_WARPS + 1;
   static constexpr int NTHREADS = 32 * (SM_WARPS + 4);
-  // register split (NQT = 2: 384 threads launch with 168 registers each =
-  // 64512; softmax warpgroups get 224, the control warpgroup keeps 56:
-  // 2*128*224 + 128*56 = 64512)
+  // register split (two softmax warpgroups: 384 threads launch with 168
+  // registers each = 64512; the softmax warpgroups get 200, the control
+  // warpgroup 104: 2*128*200 + 128*104 = 64512)
   static constexpr int REG_LAUNCH = 65536 / NTHREADS >= 255 ? 255 : (65536 / NTHREADS) / 8 * 8;
   static constexpr bool SPLIT_REGS = NQT * NS == 2;
   static constexpr int REG_SOFTMAX = 200, REG_CONTROL = 104;

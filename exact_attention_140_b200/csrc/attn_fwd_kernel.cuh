@@ -193,10 +193,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
       for (int c = 0; c < BN / 32; ++c) ptx::tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
       float m_blk;
       if (partial) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, (c < nvis) ? __uint_as_float(sr[c]) * sl2 : -INFINITY);
-        m_blk = mx;
+        m_blk = masked_max_scaled<BN>(sr, nvis, sl2);
       } else if (sl2 >= 0.f) {
         float a0 = __uint_as_float(sr[0]), a1 = __uint_as_float(sr[1]);
         float a2 = __uint_as_float(sr[2]), a3 = __uint_as_float(sr[3]);
@@ -248,21 +245,18 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
             const int col = 32 * ch + 2 * c;
             const float s0 = __uint_as_float(sr[col]), s1 = __uint_as_float(sr[col + 1]);
             float e0, e1;
-            if constexpr (PARTIAL) {
-              e0 = ptx::ex2((col < nvis ? s0 * sl2 : -INFINITY) - m_use);
-              e1 = ptx::ex2((col + 1 < nvis ? s1 * sl2 : -INFINITY) - m_use);
+            const uint64_t x = ptx::ffma2(ptx::f2(s0, s1), sl2x2, negm2);
+            float x0, x1;
+            ptx::unf2(x, x0, x1);
+            if (((16 * ch + c) % 8) < Cfg::EMU) {
+              exp2_soft2(x0, x1, e0, e1);
             } else {
-              const uint64_t x = ptx::ffma2(ptx::f2(s0, s1), sl2x2, negm2);
-              float x0, x1;
-              ptx::unf2(x, x0, x1);
-              if constexpr (true) {
-                if (((16 * ch + c) % 8) < Cfg::EMU) {
-                  exp2_soft2(x0, x1, e0, e1);
-                } else {
-                  e0 = ptx::ex2(x0);
-                  e1 = ptx::ex2(x1);
-                }
-              }
+              e0 = ptx::ex2(x0);
+              e1 = ptx::ex2(x1);
+            }
+            if constexpr (PARTIAL) {  // masked keys (a prefix is visible) get exact zeros
+              e0 = col < nvis ? e0 : 0.f;
+              e1 = col + 1 < nvis ? e1 : 0.f;
             }
             lsum[c % 4] = ptx::fadd2(lsum[c % 4], ptx::f2(e0, e1));
             if constexpr (Cfg::FP8) {

@@ -31,7 +31,12 @@
 //     item differ in length) left a tile idle for about a step per item.
 // PSEP (d = 64) gives P columns of its own (S 128 + P 64 + O 64 per tile), so
 // Q K_{j+1}^T runs during the softmax of tile j; the softmax signals s_free
-// once S is in registers and waits for the previous P V before writing P.
+// once S is in registers and waits for the previous P V before storing the
+// first chunk of P (after that chunk's exponentials, which hide the product).
+// OST (d = 64) stages each output tile in shared memory and writes it with one
+// TMA store: the rows of O are H * d elements apart, so one row per thread
+// would make every store instruction touch 32 rows; o_free is signalled as
+// soon as O has left tensor memory.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -74,7 +79,8 @@ __device__ __forceinline__ Item decode_item(int i, const FwdParams& p) {
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
     attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                               const FwdParams p) {
   constexpr int BM = Cfg::BM, BN = Cfg::BN, D = Cfg::D, NQT = Cfg::NQT, SB = Cfg::SB;
   constexpr int KST = Cfg::KST, VST = Cfg::VST;
   extern __shared__ uint8_t smem_raw[];
@@ -141,6 +147,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
     ptx::prefetch_tmap(&tmQ);
     ptx::prefetch_tmap(&tmK);
     ptx::prefetch_tmap(&tmV);
+    if constexpr (Cfg::OST) ptx::prefetch_tmap(&tmO);
   }
   if (warp == Cfg::MMA_WARP) {
     ptx::tmem_alloc(sbase + Cfg::OFF_SLOT, Cfg::TMEM_COLS);
@@ -197,10 +204,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         }
         float m_blk;
         if (partial) {
-          float mx = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < BN; ++c) mx = fmaxf(mx, (c < nvis) ? __uint_as_float(sr[c]) * sl2 : -INFINITY);
-          m_blk = mx;
+          m_blk = masked_max_scaled<BN>(sr, nvis, sl2);
         } else if (sl2 >= 0.f) {
           float a0 = __uint_as_float(sr[0]), a1 = __uint_as_float(sr[1]);
           float a2 = __uint_as_float(sr[2]), a3 = __uint_as_float(sr[3]);
@@ -230,18 +234,6 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         }
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         const bool resc_any = __any_sync(0xffffffffu, resc);
-        if constexpr (Cfg::PSEP) {
-          // P has one buffer per tile: the previous P V (product scount - 1)
-          // must have read it.  Product scount cannot have completed (its P is
-          // not written yet) and product scount - 2 was waited for one tile
-          // earlier, so the parity test is unambiguous.
-          if (scount > 0) {
-            ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_ODONE + t), (uint32_t)((scount - 1) & 1), wc, kSiteODone);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            ptx::tc_fence_after();
-          }
-        }
         const uint32_t p_taddr =
             Cfg::PSEP ? tmem_s + lane_off + (uint32_t)(Cfg::P_COL0 + t * Cfg::P_COLS) : s_taddr;
         // ---- exponentiate 32 columns at a time; each chunk's packed P is
@@ -263,19 +255,18 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
               const int col = 32 * ch + 2 * c;
               const float s0 = __uint_as_float(sr[col]), s1 = __uint_as_float(sr[col + 1]);
               float e0, e1;
-              if constexpr (PARTIAL) {
-                e0 = ptx::ex2((col < nvis ? s0 * sl2 : -INFINITY) - m_use);
-                e1 = ptx::ex2((col + 1 < nvis ? s1 * sl2 : -INFINITY) - m_use);
+              const uint64_t x = ptx::ffma2(ptx::f2(s0, s1), sl2x2, negm2);
+              float x0, x1;
+              ptx::unf2(x, x0, x1);
+              if (((16 * ch + c) % 8) < Cfg::EMU) {
+                exp2_soft2(x0, x1, e0, e1);
               } else {
-                const uint64_t x = ptx::ffma2(ptx::f2(s0, s1), sl2x2, negm2);
-                float x0, x1;
-                ptx::unf2(x, x0, x1);
-                if (((16 * ch + c) % 8) < Cfg::EMU) {
-                  exp2_soft2(x0, x1, e0, e1);
-                } else {
-                  e0 = ptx::ex2(x0);
-                  e1 = ptx::ex2(x1);
-                }
+                e0 = ptx::ex2(x0);
+                e1 = ptx::ex2(x1);
+              }
+              if constexpr (PARTIAL) {  // masked keys (a prefix is visible) get exact zeros
+                e0 = col < nvis ? e0 : 0.f;
+                e1 = col + 1 < nvis ? e1 : 0.f;
               }
               lsum[c % 4] = ptx::fadd2(lsum[c % 4], ptx::f2(e0, e1));
               if constexpr (Cfg::FP8) {
@@ -287,6 +278,22 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
                 }
               } else {
                 pk[c] = ptx::pack_bf16x2(e0, e1);
+              }
+            }
+            if constexpr (Cfg::PSEP) {
+              // P has one buffer per tile: the previous P V (product scount -
+              // 1) must have read it before the first chunk of this P is
+              // stored; the wait comes after the first chunk's exponentials,
+              // which hide most of that product.  Product scount cannot have
+              // completed (its P is not written yet) and product scount - 2
+              // was waited for one tile earlier, so the parity test is
+              // unambiguous.  A failed wait stores the rest anyway (the block
+              // is aborting; the addresses are its own) and leaves the loop
+              // after this tile.
+              if (ch == 0 && scount > 0) {
+                ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_ODONE + t), (uint32_t)((scount - 1) & 1), wc, kSiteODone);
+                ok = __all_sync(0xffffffffu, ok);
+                ptx::tc_fence_after();
               }
             }
             if constexpr (Cfg::FP8)
@@ -307,6 +314,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
           exp_row(std::true_type{});
         else
           exp_row(std::false_type{});
+        if (!ok) break;
         {
           float la, lb;
           ptx::unf2(ptx::fadd2(ptx::fadd2(lsum[0], lsum[1]), ptx::fadd2(lsum[2], lsum[3])), la, lb);
@@ -340,48 +348,96 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         if (resc_any) ptx::mbar_arrive(bar(Cfg::B_PHALF + si));
         ptx::mbar_arrive(bar(Cfg::B_PFULL + si));
       }
-      if (!ok) break;
+      if (!Cfg::OST && !ok) break;
       // ---------------------------------------------------------- epilogue
-      if (nt > 0) {  // o_final completes once per item, after the tile's last PV
+      if (ok && nt > 0) {  // o_final completes once per item, after the tile's last PV
         ok = wait_bar<kRoleSoftmax>(bar(Cfg::B_OFINAL + t), (uint32_t)(finals & 1), wc, kSiteODone);
         ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        ++finals;
+        if (ok) ++finals;
       }
+      if constexpr (Cfg::OST) {
+        // The staging tile is free once the previous item's store has read
+        // it.  The four warps of the stream meet at this named barrier on
+        // every item, failed waits included, and leave together.
+        if (wq == 0 && lane == 0) ptx::bulk_wait_read0();
+        ok = ptx::bar_red_and(1u + (uint32_t)s, 128u, ok);
+      }
+      if (!ok) break;
       ptx::tc_fence_after();
       const bool store = row < p.Nq;
       float inv = l > 0.f ? 1.f / l : 0.f;
       if constexpr (Cfg::FP8) inv *= __ldg(p.dv);
       const Item ie = decode_item(item, p);  // recomputed: keeps fewer values live through the key loop
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                            (((long long)ie.b * p.Nq + row) * p.Hq + ie.h) * (long long)D;
+      if constexpr (Cfg::OST) {
+        // row r of the tile -> 128-byte row r of the staging tile, 16-byte
+        // unit u at position u ^ (r % 8) (the 128-byte swizzle of the map)
+        const uint32_t ost = sstream + Cfg::OFF_OST;
+        const uint32_t r = (uint32_t)(wq * 32 + lane);
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        if (nt > 0) {
-          ptx::tmem_ld32(o_taddr + 32 * c, r);
-          ptx::tmem_wait_ld_dep(r);
-        }
-        uint32_t w[16];
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rr[32];
+          if (nt > 0) {
+            ptx::tmem_ld32(o_taddr + 32 * c, rr);
+            ptx::tmem_wait_ld_dep(rr);
+          }
+          uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = nt > 0 ? ptx::pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv)
-                        : 0u;
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+          for (int e = 0; e < 16; ++e)
+            w[e] = nt > 0 ? ptx::pack_bf16x2(__uint_as_float(rr[2 * e]) * inv, __uint_as_float(rr[2 * e + 1]) * inv)
+                          : 0u;
+          const uint32_t rbase = ost + (uint32_t)(c / 2) * (uint32_t)(BM * 128) + r * 128u;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          for (int e = 0; e < 4; ++e)
+            ptx::st_shared_v4(rbase + ((((uint32_t)(c & 1) * 4u + (uint32_t)e) ^ (r & 7u)) << 4), w[4 * e],
+                              w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
         }
-      }
-      if (nt > 0) {  // O of this tile is read out: the next item may overwrite it
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(Cfg::B_OFREE + t));
+        if (nt > 0) {  // O of this tile is read out: the next item may overwrite it
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bar(Cfg::B_OFREE + t));
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::bar_sync(1u + (uint32_t)s, 128u);
+        if (wq == 0 && lane == 0) {
+          // rows at or past Nq fall outside the map and are not written
+#pragma unroll
+          for (int cb = 0; cb < Cfg::NCH; ++cb)
+            ptx::tma_store_4d(&tmO, ost + (uint32_t)cb * (uint32_t)(BM * 128), cb * 64, ie.h, row0, ie.b);
+          ptx::bulk_commit();
+        }
+      } else {
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
+                              (((long long)ie.b * p.Nq + row) * p.Hq + ie.h) * (long long)D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          if (nt > 0) {
+            ptx::tmem_ld32(o_taddr + 32 * c, r);
+            ptx::tmem_wait_ld_dep(r);
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = nt > 0 ? ptx::pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv)
+                          : 0u;
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
+        }
+        if (nt > 0) {  // O of this tile is read out: the next item may overwrite it
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bar(Cfg::B_OFREE + t));
+        }
       }
       if (store && p.lse != nullptr) {
         const float lse = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
         p.lse[((long long)ie.b * p.Hq + ie.h) * p.Nq + row] = lse;
       }
     }
+    // the staging tile's last store must be complete before the block exits
+    if constexpr (Cfg::OST)
+      if (wq == 0 && lane == 0) ptx::bulk_wait0();
   } else if (is_tma) {
     // ------------------------------------------------------------ producer
     constexpr int kProducerRole = Cfg::NS > 1 ? kRoleProducerBackoff : kRoleProducer;

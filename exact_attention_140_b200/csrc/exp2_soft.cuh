@@ -12,7 +12,7 @@
 //   exact.  2^j is applied by adding j << 23 to the bits of p(f); with
 //   j >= -125 the result stays a normal float.  Results below 2^-125 (the
 //   clamp) are returned as about 2^-125 instead of 0; callers that need exact
-//   zeros (masked keys) use the hardware path.
+//   zeros (masked keys) select them after the call.
 #pragma once
 #include <cstdint>
 
