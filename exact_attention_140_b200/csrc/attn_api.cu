@@ -526,9 +526,13 @@ bool use_persistent(int Nk, int d, bool causal) { return Nk <= kPersistentMaxNk 
 // short-range one (persistent).  EMU is the share of softmax exponentials
 // computed in software (out of 8 element pairs), chosen by measurement.
 //   d = 64 short: two independent streams of one 128-row query tile each; P
-//   in columns of its own (S 128 + P 64 + O 64 = 256 columns per stream).
+//   in columns of its own (S 128 + P 64 + O 64 = 256 columns per stream);
+//   each output tile staged in shared memory for one TMA store (K ring of 2
+//   and V ring of 3 stages leave room for it); every exponential on the
+//   hardware unit (a software share measured slower at d = 64, where the
+//   exponentials are a small part of a key tile's time).
 template <bool C> using CfgD64 = FwdCfg<64, 128, 2, 3, 3, C, false, 3>;
-template <bool C> using CfgD64Short = FwdCfg<64, 128, 1, 2, 3, C, false, 2, 1, true, 2, false, true>;
+template <bool C> using CfgD64Short = FwdCfg<64, 128, 1, 2, 3, C, false, 0, 1, true, 2, false, true>;
 template <bool C> using CfgD128 = FwdCfg<128, 128, 2, 2, 2, C, false, C ? 2 : 1>;
 template <bool C> using CfgD128Short = FwdCfg<128, 128, 2, 2, 2, C, false, 0>;
 template <bool C> using CfgD256 = FwdCfg<256, 64, 1, 2, 2, C, false, 0>;
