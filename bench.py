@@ -360,19 +360,33 @@ def run_ours(args, cfg, name):
     if rc != 0:
         raise RuntimeError(f"device error word {word:#x}")
 
-    # end to end through the C ABI with host buffers: H2D inputs, kernel(s), D2H outputs
+    # end to end with host buffers: H2D inputs, kernel(s), D2H outputs.  The bf16
+    # forward goes through attn_fwd_host (the C ABI's host-buffer entry point,
+    # which pipelines the copies and kernels over chunks of heads); the FP8 and
+    # split-KV lines copy around their device entry points.
     e2e_steps = max(3, min(args.steps, 50))
     e_st = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
     e_en = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
     dq, dk, dv = (torch.empty_like(x) for x in (q, k, v))
-    for i in range(e2e_steps):
-        e_st[i].record(stream)
+    host_path = not fp8 and not cfg.get("split")
+
+    def e2e_step():
+        if host_path:
+            ea.attn_fwd_host(host[0], host[1], host[2], o_host, lse_host, dq, dk, dv, o, lse, B, Hq, Hkv, Nq, N, d,
+                             causal, scale, 0, stream)
+            return
         dq.copy_(host[0], non_blocking=True)
         dk.copy_(host[1], non_blocking=True)
         dv.copy_(host[2], non_blocking=True)
         step(dq, dk, dv)
         o_host.copy_(o, non_blocking=True)
         lse_host.copy_(lse, non_blocking=True)
+
+    e2e_step()  # first call creates the pipeline's streams and events
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        e_st[i].record(stream)
+        e2e_step()
         e_en[i].record(stream)
     torch.cuda.synchronize()
     e2e_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_st, e_en)))
@@ -413,7 +427,9 @@ def run_ours(args, cfg, name):
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in host)),
-                "d2h_bytes_per_step": int(o.numel() * o.element_size() + lse.numel() * lse.element_size())},
+                "d2h_bytes_per_step": int(o.numel() * o.element_size() + lse.numel() * lse.element_size()),
+                "api": ("attn_fwd_host (pinned host buffers, copies and kernels pipelined over 8 chunks)"
+                        if host_path else "pinned-host copies around the device entry point")},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }

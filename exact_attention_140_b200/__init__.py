@@ -21,7 +21,7 @@ __all__ = [
     "attn_kv_tile_count", "attn_tile_kind", "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attention",
     "attn_fwd_schedule", "attn_hadamard_quant_fp8_noalloc", "attn_fwd_splitkv", "attn_splitkv_workspace_bytes",
     "attn_combine", "attn_kv_tile_count_window", "attn_tile_kind_window", "attn_gemm_add", "lib_path", "EXPORTS",
-    "attn_debug_map_cache_stats", "attn_fwd_part", "attn_shard_units", "attention_shard",
+    "attn_debug_map_cache_stats", "attn_fwd_part", "attn_shard_units", "attention_shard", "attn_fwd_host",
 ]
 
 ATTN_BF16 = 0
@@ -39,6 +39,7 @@ EXPORTS = (
     "attn_debug_unsatisfied_wait", "attn_debug_exp2", "attn_hadamard_quant_fp8_noalloc", "attn_fwd_schedule",
     "attn_fwd_splitkv", "attn_splitkv_workspace_bytes", "attn_combine", "attn_kv_tile_count_window",
     "attn_tile_kind_window", "attn_gemm_add", "attn_debug_map_cache_stats", "attn_fwd_part", "attn_shard_units",
+    "attn_fwd_host",
 )
 
 if not os.path.exists(lib_path):
@@ -52,6 +53,8 @@ _lib.attn_fwd.restype = _I
 _lib.attn_fwd_part.argtypes = [_vp] * 5 + [_I] * 7 + [_F, _I] + [_I] * 4 + [_vp]
 _lib.attn_fwd_part.restype = _I
 _lib.attn_shard_units.argtypes = [_I] * 4 + [ctypes.POINTER(_I)]
+_lib.attn_fwd_host.argtypes = [_vp] * 10 + [_I] * 7 + [_F, _I, _vp]
+_lib.attn_fwd_host.restype = _I
 _lib.attn_shard_units.restype = _I
 _lib.attn_fwd_fp8.argtypes = [_vp] * 5 + [_I] * 7 + [_F, _vp, _vp, _vp, _vp]
 _lib.attn_fwd_fp8.restype = _I
@@ -137,6 +140,17 @@ def attn_fwd_part(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype, 
                             float(scale), int(dtype), int(b_begin), int(b_end), int(kvh_begin), int(kvh_end),
                             _stream(stream))
     return _check(rc, "attn_fwd_part", raise_on_error)
+
+
+def attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                  n_chunks=0, stream=None, raise_on_error=True):
+    """attn_fwd with host inputs/outputs (pinned for overlap) and caller-owned
+    device buffers; the copies in, kernels and copies out are pipelined over
+    n_chunks runs of (batch, key/value head) units (0: the library's default)."""
+    rc = _lib.attn_fwd_host(_ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(o_h), _ptr(lse_h), _ptr(q_d), _ptr(k_d),
+                            _ptr(v_d), _ptr(o_d), _ptr(lse_d), B, Hq, Hkv, Nq, Nk, d, int(causal), float(scale),
+                            int(n_chunks), _stream(stream))
+    return _check(rc, "attn_fwd_host", raise_on_error)
 
 
 def attn_shard_units(B, Hkv, world, rank):

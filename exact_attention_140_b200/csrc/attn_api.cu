@@ -56,6 +56,30 @@ using CtxGetCurrentFn = CUresult (*)(CUcontext*);
 EncodeTiledFn g_encode = nullptr;
 CtxGetCurrentFn g_ctx_current = nullptr;
 
+// ATTN_LOG=1 in the environment: every launch prints its kernel, template
+// configuration, grid and problem size to stderr (read once; silent otherwise).
+bool log_on() {
+  static const bool v = [] {
+    const char* e = std::getenv("ATTN_LOG");
+    return e != nullptr && std::atoi(e) > 0;
+  }();
+  return v;
+}
+#define ATTN_LOGF(...)                        \
+  do {                                        \
+    if (log_on()) std::fprintf(stderr, __VA_ARGS__); \
+  } while (0)
+template <class Cfg>
+void log_launch(const char* kernel, dim3 grid, int B, int Hq, int Hkv, int Nq, int Nk, const char* extra = "") {
+  if (!log_on()) return;
+  std::fprintf(stderr,
+               "attn: %s<D=%d BN=%d NQT=%d KST=%d VST=%d causal=%d fp8=%d EMU=%d SB=%d PSEP=%d NS=%d OST=%d> "
+               "grid=(%u,%u,%u) block=%d smem=%u B=%d Hq=%d Hkv=%d Nq=%d Nk=%d%s\n",
+               kernel, Cfg::D, Cfg::BN, Cfg::NQT, Cfg::KST, Cfg::VST, (int)Cfg::CAUSAL, (int)Cfg::FP8, Cfg::EMU, Cfg::SB,
+               (int)Cfg::PSEP, Cfg::NS, (int)Cfg::OST, grid.x, grid.y, grid.z, Cfg::NTHREADS, Cfg::SMEM_BYTES, B, Hq,
+               Hkv, Nq, Nk, extra);
+}
+
 unsigned long long timeout_ns() {
   static unsigned long long v = [] {
     const char* e = std::getenv("ATTN_WAIT_TIMEOUT_NS");
@@ -388,6 +412,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.band = (int)band;
     grid = dim3((unsigned)p.n_items, 1u, 1u);
   }
+  log_launch<Cfg>("attn_fwd_kernel", grid, B, Hq, Hkv, Nq, Nk, Cfg::CAUSAL ? " (1-D grid, head bands)" : "");
   attn_fwd_kernel<Cfg><<<grid, Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -409,6 +434,7 @@ int launch_fwd_persistent(const void* q, const void* k, const void* v, void* o, 
   if (Cfg::OST && encode_bnhd(&to, o, false, B, Nq, Hq, Cfg::D, Cfg::BM) != ATTN_OK) return ATTN_ERR_CUDA;
   const int nstreams = (p.n_items + Cfg::NS - 1) / Cfg::NS;  // blocks that find work
   const int nblk = nstreams < st->num_sms ? nstreams : st->num_sms;
+  log_launch<Cfg>("attn_fwd_persistent_kernel", dim3((unsigned)nblk), B, Hq, Hkv, Nq, Nk);
   attn_fwd_persistent_kernel<Cfg><<<dim3((unsigned)nblk), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -436,6 +462,11 @@ int launch_fwd_split(const void* q, const void* k, const void* v, float* o_part,
   p.pack = pack;
   if (pack > 1) p.n_qblocks = (int)(((long long)Nq * pack + Cfg::BM * Cfg::NQT - 1) / (Cfg::BM * Cfg::NQT));
   const dim3 grid((unsigned)p.n_qblocks, (unsigned)(pack > 1 ? Hkv : Hq), (unsigned)(B * n_splits));
+  if (log_on()) {
+    char extra[64];
+    std::snprintf(extra, sizeof extra, " split-KV windows=%d chunk=%d pack=%d", n_splits, kv_chunk, pack);
+    log_launch<Cfg>("attn_fwd_kernel", grid, B, Hq, Hkv, Nq, Nk, extra);
+  }
   attn_fwd_kernel<Cfg><<<grid, Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -473,6 +504,8 @@ int launch_combine(const float* o_part, const float* lse_part, int S, int B, int
   const long long blocks = (rows * 32 + 255) / 256;
   if (blocks > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
   auto* ob = reinterpret_cast<__nv_bfloat16*>(o);
+  ATTN_LOGF("attn: attn_combine_kernel<%d> grid=(%lld) block=256 windows=%d B=%d Hq=%d Nq=%d\n", d, blocks, S, B, Hq,
+            Nq);
   switch (d) {
     case 64: attn_combine_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(o_part, lse_part, S, B, Hq, Nq, ob, lse); break;
     case 128: attn_combine_kernel<128><<<(unsigned)blocks, 256, 0, s>>>(o_part, lse_part, S, B, Hq, Nq, ob, lse); break;
@@ -583,6 +616,8 @@ int launch_prep_passes(const CUtensorMap& tx, const CUtensorMap& tx8, const Prep
                                                                         : PrepCfg<false>::BLOCKS_PER_SM * st->num_sms;
   const int gq = p.n_tiles < PrepCfg<true>::BLOCKS_PER_SM * st->num_sms ? p.n_tiles
                                                                        : PrepCfg<true>::BLOCKS_PER_SM * st->num_sms;
+  ATTN_LOGF("attn: fp8_prep_kernel<rotate=%d> amax pass grid=(%d) + quantising pass grid=(%d) block=%d rows=%lld\n",
+            (int)ROT, ga, gq, kPrepRows, (long long)p.rows);
   fp8_prep_kernel<ROT, false><<<ga, kPrepRows, PrepCfg<false>::SMEM_BYTES, s>>>(tx, tx8, p);
   fp8_prep_kernel<ROT, true><<<gq, kPrepRows, PrepCfg<true>::SMEM_BYTES, s>>>(tx, tx8, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -682,6 +717,49 @@ int shard_rects(int B, int Hkv, int world, int rank, int* r) {
   return n;
 }
 
+// Streams and events of the host-buffer pipeline (attn_fwd_host), one set per
+// device, created at the first call in the device's current context and
+// rebuilt when the context changes (the old handles died with it).  The
+// events are shared by successive calls: each call enqueues under the
+// device's pipeline mutex, and a stream wait binds to the record made just
+// before it, so a later call re-recording an event cannot disturb an earlier
+// call's dependencies.
+constexpr int kMaxChunks = 64;
+struct Pipe {
+  CUcontext ctx = nullptr;
+  cudaStream_t in = nullptr, out = nullptr;  // host-to-device and device-to-host copies
+  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t in_done[kMaxChunks] = {}, comp_done[kMaxChunks] = {};
+};
+Pipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mu[kMaxDevices];
+
+int pipe_get(int dev, const DeviceState* st, Pipe** out) {
+  Pipe& pp = g_pipe[dev];
+  if (pp.ctx != st->ctx) {
+    Pipe fresh;
+    auto ev = [](cudaEvent_t* e) { return cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess; };
+    bool ok = cudaStreamCreateWithFlags(&fresh.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&fresh.out, cudaStreamNonBlocking) == cudaSuccess && ev(&fresh.start) &&
+              ev(&fresh.end);
+    for (int c = 0; ok && c < kMaxChunks; ++c) ok = ev(&fresh.in_done[c]) && ev(&fresh.comp_done[c]);
+    if (!ok) return ATTN_ERR_CUDA;
+    fresh.ctx = st->ctx;
+    pp = fresh;
+  }
+  *out = &pp;
+  return ATTN_OK;
+}
+
+// One strided block of rows between host and device: `rows` rows of `width`
+// bytes, `pitch` bytes apart in both buffers, starting `off` bytes in.
+cudaError_t copy_rows(void* dst, const void* src, size_t off, size_t width, size_t pitch, size_t rows,
+                      cudaMemcpyKind kind, cudaStream_t s) {
+  if (width == 0 || rows == 0) return cudaSuccess;
+  return cudaMemcpy2DAsync(static_cast<char*>(dst) + off, pitch, static_cast<const char*>(src) + off, pitch, width,
+                           rows, kind, s);
+}
+
 }  // namespace
 }  // namespace attn
 
@@ -746,6 +824,79 @@ int attn_fwd_part(const void* q, const void* k, const void* v, void* o, float* l
 int attn_shard_units(int B, int Hkv, int world, int rank, int* rects) {
   if (B < 0 || Hkv < 0 || world < 1 || rank < 0 || rank >= world || rects == nullptr) return -1;
   return shard_rects(B, Hkv, world, rank, rects);
+}
+
+int attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, float* lse_h, void* q_d, void* k_d,
+                  void* v_d, void* o_d, float* lse_d, int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                  float scale, int n_chunks, void* stream) {
+  if (q_h == nullptr || o_h == nullptr || (Nk > 0 && (k_h == nullptr || v_h == nullptr)) || n_chunks < 0 ||
+      (lse_h != nullptr && lse_d == nullptr))
+    return ATTN_ERR_INVALID_ARG;
+  int rc = check_common(q_d, k_d, v_d, o_d, lse_d, B, Hq, Hkv, Nq, Nk, causal, scale);
+  if (rc == -1) return ATTN_OK;
+  if (rc != ATTN_OK) return rc;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  int dev = 0;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&dev, &st)) != ATTN_OK) return rc;
+  std::lock_guard<std::mutex> lk(g_pipe_mu[dev]);
+  Pipe* pp = nullptr;
+  if ((rc = pipe_get(dev, st, &pp)) != ATTN_OK) return rc;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long units = (long long)B * Hkv;
+  long long nc = n_chunks == 0 ? 8 : n_chunks;
+  nc = nc > units ? units : nc;
+  nc = nc > kMaxChunks ? kMaxChunks : nc;
+  const int C = (int)nc, g = Hq / Hkv;
+  const size_t es = 2;  // bf16
+  const size_t qpitch = (size_t)Hq * d * es, kpitch = (size_t)Hkv * d * es, lpitch = (size_t)Hq * Nq * 4;
+#define ATTN_CK(x)                                   \
+  do {                                               \
+    if ((x) != cudaSuccess) return ATTN_ERR_CUDA; \
+  } while (0)
+  // the copies start after the work already on `stream`
+  ATTN_CK(cudaEventRecord(pp->start, s));
+  ATTN_CK(cudaStreamWaitEvent(pp->in, pp->start, 0));
+  ATTN_CK(cudaStreamWaitEvent(pp->out, pp->start, 0));
+  for (int c = 0; c < C; ++c) {
+    int r[12];
+    const int nr = shard_rects(B, Hkv, C, c, r);
+    for (int i = 0; i < nr; ++i) {  // in: this chunk's heads of every row of Q, K, V
+      const size_t b0 = (size_t)r[4 * i], nb = (size_t)(r[4 * i + 1] - r[4 * i]);
+      const size_t g0 = (size_t)r[4 * i + 2], ng = (size_t)(r[4 * i + 3] - r[4 * i + 2]);
+      ATTN_CK(copy_rows(q_d, q_h, (b0 * Nq * Hq + g0 * g) * d * es, ng * g * d * es, qpitch, nb * Nq,
+                        cudaMemcpyHostToDevice, pp->in));
+      if (Nk > 0) {
+        const size_t koff = (b0 * Nk * Hkv + g0) * d * es;
+        ATTN_CK(copy_rows(k_d, k_h, koff, ng * d * es, kpitch, nb * Nk, cudaMemcpyHostToDevice, pp->in));
+        ATTN_CK(copy_rows(v_d, v_h, koff, ng * d * es, kpitch, nb * Nk, cudaMemcpyHostToDevice, pp->in));
+      }
+    }
+    ATTN_CK(cudaEventRecord(pp->in_done[c], pp->in));
+    ATTN_CK(cudaStreamWaitEvent(s, pp->in_done[c], 0));
+    for (int i = 0; i < nr; ++i) {
+      const Part pt{r[4 * i], r[4 * i + 1] - r[4 * i], r[4 * i + 2] * g, (r[4 * i + 3] - r[4 * i + 2]) * g};
+      if ((rc = fwd_checked(q_d, k_d, v_d, o_d, lse_d, B, Hq, Hkv, Nq, Nk, d, causal != 0, scale, false, nullptr,
+                            nullptr, nullptr, pt, st, s)) != ATTN_OK)
+        return rc;
+    }
+    ATTN_CK(cudaEventRecord(pp->comp_done[c], s));
+    ATTN_CK(cudaStreamWaitEvent(pp->out, pp->comp_done[c], 0));
+    for (int i = 0; i < nr; ++i) {  // out: this chunk's O rows (and LSE entries)
+      const size_t b0 = (size_t)r[4 * i], nb = (size_t)(r[4 * i + 1] - r[4 * i]);
+      const size_t g0 = (size_t)r[4 * i + 2], ng = (size_t)(r[4 * i + 3] - r[4 * i + 2]);
+      ATTN_CK(copy_rows(o_h, o_d, (b0 * Nq * Hq + g0 * g) * d * es, ng * g * d * es, qpitch, nb * Nq,
+                        cudaMemcpyDeviceToHost, pp->out));
+      if (lse_h != nullptr)
+        ATTN_CK(copy_rows(lse_h, lse_d, (b0 * Hq + g0 * g) * Nq * 4, ng * g * Nq * 4, lpitch, nb,
+                          cudaMemcpyDeviceToHost, pp->out));
+    }
+  }
+  // `stream` completes only after the last copy out
+  ATTN_CK(cudaEventRecord(pp->end, pp->out));
+  ATTN_CK(cudaStreamWaitEvent(s, pp->end, 0));
+#undef ATTN_CK
+  return ATTN_OK;
 }
 
 int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
@@ -896,6 +1047,8 @@ int attn_gemm_add(const void* a, const void* b, const void* c, void* d, int M, i
   p.err = st->err;
   p.timeout_ns = timeout_ns();
   const int nblk = p.n_tiles < st->num_sms ? p.n_tiles : st->num_sms;
+  ATTN_LOGF("attn: gemm_add_kernel grid=(%d) block=%d smem=%u M=%d N=%d K=%d C=%s tiles=%d\n", nblk, GemmCfg::NTHREADS,
+            (unsigned)GemmCfg::SMEM_BYTES, M, N, K, c != nullptr ? "yes" : "no", p.n_tiles);
   gemm_add_kernel<<<dim3((unsigned)nblk), GemmCfg::NTHREADS, GemmCfg::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
       ta, tb, tc, td, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

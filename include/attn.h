@@ -41,6 +41,14 @@
  * Threads:   all entry points are thread-safe.
  * Empty:     B == 0, Hq == 0 or Nq == 0 is a no-op returning ATTN_OK.  Nk == 0
  *            gives O = 0 and LSE = -inf for every row.
+ * Environment (read once, at the first call):
+ *            ATTN_LOG=1 prints one line per kernel launch to stderr: the
+ *            kernel, its template configuration (head size, key tile, query
+ *            tiles per block, ring stages, causal, dtype, software-exp share,
+ *            score buffers, separate P, streams, staged output), grid, block,
+ *            shared memory and problem size.  The library is silent otherwise.
+ *            ATTN_WAIT_TIMEOUT_NS=<n> sets the limit of every device-side wait
+ *            in nanoseconds (default 2 s).
  */
 #ifndef LIBATTN_ATTN_H_
 #define LIBATTN_ATTN_H_
@@ -113,6 +121,42 @@ int attn_fwd_part(const void *q, const void *k, const void *v, void *o, float *l
  * Host-only; no CUDA call.
  */
 int attn_shard_units(int B, int Hkv, int world, int rank, int *rects);
+
+/*
+ * attn_fwd_host -- attn_fwd (bf16) with its inputs and outputs in HOST memory:
+ * the call copies Q, K and V in, computes, and copies O (and LSE) out, all
+ * enqueued on `stream`.  The work is cut into n_chunks runs of the B * Hkv
+ * (batch, key/value head) units (the split of attn_shard_units, so a
+ * grouped-query group stays whole) and pipelined: the copies in of chunk
+ * c + 1 and the copies out of chunk c - 1 run while chunk c computes.  The
+ * copies run on two streams of the library's own (one per direction), made to
+ * wait for the work already on `stream` and joined back to it, so the host
+ * outputs are complete when `stream` is.  Each chunk moves strided rows (its
+ * heads of every sequence row) with one 2-D copy per tensor and rectangle.
+ *   q_h, k_h, v_h    host inputs, layouts as attn_fwd.  Page-locked memory
+ *                    (cudaHostAlloc, cudaHostRegister, torch pin_memory) lets
+ *                    the copies overlap; pageable memory works but serialises.
+ *   o_h, lse_h       host outputs; lse_h may be NULL (then LSE stays on the
+ *                    device, if lse_d is given, or is not computed).
+ *   q_d, k_d, v_d, o_d, lse_d
+ *                    caller-owned DEVICE buffers of the full tensors, as for
+ *                    attn_fwd (16-byte aligned; lse_d may be NULL only when
+ *                    lse_h is NULL).  They hold the inputs and results after
+ *                    the call as attn_fwd's tensors would.
+ *   n_chunks         pipeline depth, >= 1; 0 picks 8.  Clamped to B * Hkv.
+ *   B, Hq, Hkv, Nq, Nk, d, causal, scale, stream   as attn_fwd.
+ * Host buffers must not overlap the device ones.  The library allocates no
+ * memory for the data; its two streams and a few events per device are
+ * created at the first call and kept.  Calls from several host threads are
+ * serialised while they enqueue.  Returns as attn_fwd (ATTN_ERR_INVALID_ARG
+ * also for a NULL host pointer, n_chunks < 0, or lse_h without lse_d);
+ * ATTN_ERR_CUDA if an enqueue fails part way (the stream may then hold part
+ * of the work).
+ */
+int attn_fwd_host(const void *q_h, const void *k_h, const void *v_h, void *o_h, float *lse_h,
+                  void *q_d, void *k_d, void *v_d, void *o_d, float *lse_d,
+                  int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                  int n_chunks, void *stream);
 
 /*
  * attn_fwd_fp8 -- FP8 E4M3 attention forward with per-tensor scales.

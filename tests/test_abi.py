@@ -229,3 +229,26 @@ def test_fwd_part_range_errors_before_any_cuda_call():
     assert part(0, 2, 0, 5) == INVALID
     assert part(0, 2, 0, 4, d=96) == UNSUPPORTED
     assert part(0, 2, 0, 4, Nq=0) == OK  # nothing to compute
+
+
+def test_fwd_host_argument_errors_before_any_cuda_call():
+    host = np.zeros(16, dtype=np.uint8)  # stands in for every host buffer; never touched
+    H = host.ctypes.data
+
+    def call(q_h=H, k_h=H, v_h=H, o_h=H, lse_h=None, lse_d=None, n_chunks=0, **kw):
+        a = dict(B=2, Hq=8, Hkv=4, Nq=64, Nk=64, d=128, causal=0, scale=0.1)
+        a.update(kw)
+        return ea.attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, FAKE, FAKE, FAKE, FAKE, lse_d, a["B"], a["Hq"], a["Hkv"],
+                                a["Nq"], a["Nk"], a["d"], a["causal"], a["scale"], n_chunks=n_chunks, stream=0,
+                                raise_on_error=False)
+    assert call(q_h=None) == INVALID
+    assert call(o_h=None) == INVALID
+    assert call(k_h=None) == INVALID
+    assert call(v_h=None) == INVALID
+    assert call(n_chunks=-1) == INVALID
+    assert call(lse_h=H) == INVALID            # a host LSE needs a device LSE buffer
+    assert call(Hq=6) == INVALID               # Hq % Hkv != 0
+    assert call(scale=float("nan")) == INVALID
+    assert call(d=96) == UNSUPPORTED
+    assert call(B=0) == OK                     # nothing to compute
+    assert call(Nq=0) == OK
