@@ -190,13 +190,33 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         const uint32_t s_taddr = tmem_s + lane_off + (uint32_t)(si * BN);
         const bool partial = tile_kind(row0, row0 + BM, j, p.Nq, p.Nk, BN, Cfg::CAUSAL) == kTilePartial;
         const int nvis = vend - j * BN;  // visible keys of this tile (masks partial tiles)
-        // ---- one read of the whole score row (one TMEM load latency per tile)
+        // ---- one read of the whole score row per tile, in two halves: the
+        // second half's loads are in flight while the first half's maximum is
+        // taken (full tiles, scale >= 0)
         uint32_t sr[BN];
+        constexpr int NCH = BN / 32, NCH0 = NCH / 2 > 0 ? NCH / 2 : 1;
+        const bool fast_max = !partial && sl2 >= 0.f;
+        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
+        for (int c = 0; c < NCH0; ++c)
           ptx::tmem_ld32(s_taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) ptx::tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+        for (int c = 0; c < NCH0; ++c) ptx::tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+#pragma unroll
+        for (int c = NCH0; c < NCH; ++c)
+          ptx::tmem_ld32(s_taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+        auto fold = [&](int c0, int c1) {  // a0..a3 <- their max with scores [c0, c1)
+#pragma unroll
+          for (int c = c0; c < c1; c += 8) {
+            a0 = ptx::fmax3(a0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+            a1 = ptx::fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+            a2 = ptx::fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+            a3 = ptx::fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+          }
+        };
+        if (fast_max) fold(0, 32 * NCH0);
+#pragma unroll
+        for (int c = NCH0; c < NCH; ++c) ptx::tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
         if constexpr (Cfg::PSEP) {
           // S is in registers: the next Q K^T of this tile may overwrite it
           ptx::tc_fence_before();
@@ -206,17 +226,7 @@ __global__ void __launch_bounds__(Cfg::NTHREADS, 1)
         if (partial) {
           m_blk = masked_max_scaled<BN>(sr, nvis, sl2);
         } else if (sl2 >= 0.f) {
-          float a0 = __uint_as_float(sr[0]), a1 = __uint_as_float(sr[1]);
-          float a2 = __uint_as_float(sr[2]), a3 = __uint_as_float(sr[3]);
-#pragma unroll
-          for (int c = 4; c < BN; c += 8) {
-            a0 = ptx::fmax3(a0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-            a1 = ptx::fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-            if (c + 4 < BN) {
-              a2 = ptx::fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-              a3 = ptx::fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
-            }
-          }
+          fold(32 * NCH0, BN);
           m_blk = ptx::fmax3(a0, a1, fmaxf(a2, a3)) * sl2;
         } else {  // a negative scale turns the row max into the row min
           float mn = __uint_as_float(sr[0]);
